@@ -1,0 +1,144 @@
+// Row-wise kernels between and after the grouped GEMMs: the FP8 requantisation of the SwiGLU
+// intermediate (per routed row, over all F), the routing-weighted combine that restores token
+// order, and the reduction of K-split partials for the split entry point. All are HBM-bound:
+// 128-bit loads/stores, one block (or warp) per row, grids sized in multiples of the SM count.
+//
+// Method: megakernel page (seventnews.com), W8A8 paragraph -- FP8 activations, here also for the
+// expert intermediate; "Routage MoE entre GPU" (viite.ai) -- outputs weighted by their routing
+// weights, summed, and put back in the original token order.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+// s2[r] = amax[r] / 448 (IEEE fp32; 1 if 0); aq[r, f] = e4m3_rne_satfinite(act[r, f] / s2[r]).
+__global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ act,
+                                                      const uint32_t* __restrict__ amax,
+                                                      const int32_t* __restrict__ total_rows,
+                                                      int64_t rcap, int F,
+                                                      uint8_t* __restrict__ aq,
+                                                      float* __restrict__ s2) {
+  const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
+  const int nv = F / 4;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    const float am = __uint_as_float(amax[r]);
+    const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+    if (threadIdx.x == 0) s2[r] = sc;
+    const float4* src = reinterpret_cast<const float4*>(act + (size_t)r * F);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(aq + (size_t)r * F);
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+      const float4 v = src[i];
+      dst[i] = static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.x, sc), __fdiv_rn(v.y, sc))) |
+               (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.z, sc), __fdiv_rn(v.w, sc))) << 16);
+    }
+  }
+}
+
+// y[t, :] = bf16_rne( sum_j w[t, j] * (sum_s o[s][inv[t, j], :]) + sum_s shared[s][row0 + t, :] )
+// Slots with inv < 0 are skipped; fp32, slot order and split order fixed (deterministic).
+__global__ void __launch_bounds__(256) combine_kernel(
+    const float* __restrict__ o, int splits, size_t split_stride, const float* __restrict__ topk_w,
+    const int32_t* __restrict__ inv_row, int k_max, int64_t rcap,
+    const float* __restrict__ shared_src, const int32_t* __restrict__ shared_row0,
+    int shared_splits, size_t shared_split_stride, int T, int d, uint16_t* __restrict__ y,
+    float* __restrict__ y_f32, int* status) {
+  __shared__ int rows[kMaxK];
+  __shared__ float wts[kMaxK];
+  const int nv = d / 4;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < k_max) {
+      int r = inv_row[(size_t)t * k_max + threadIdx.x];
+      if (r >= rcap) {
+        report(status, kStatusDeviceCheck, kWhereCombine, t);
+        r = -1;
+      }
+      rows[threadIdx.x] = r;
+      wts[threadIdx.x] = topk_w[(size_t)t * k_max + threadIdx.x];
+    }
+    __syncthreads();
+    const int64_t srow = shared_src ? (int64_t)(shared_row0 ? *shared_row0 : 0) + t : -1;
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < k_max; ++j) {
+        const int r = rows[j];
+        if (r < 0) continue;
+        float4 v = reinterpret_cast<const float4*>(o + (size_t)r * d)[i];
+        for (int s = 1; s < splits; ++s) {
+          const float4 u = reinterpret_cast<const float4*>(o + s * split_stride + (size_t)r * d)[i];
+          v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+        }
+        const float w = wts[j];
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
+      }
+      if (srow >= 0) {
+        for (int s = 0; s < shared_splits; ++s) {
+          const float4 u = reinterpret_cast<const float4*>(
+              shared_src + s * shared_split_stride + (size_t)srow * d)[i];
+          acc.x += u.x; acc.y += u.y; acc.z += u.z; acc.w += u.w;
+        }
+      }
+      const uint32_t lo = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.x))) |
+                          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.y))) << 16);
+      const uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.z))) |
+                          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.w))) << 16);
+      reinterpret_cast<uint2*>(y + (size_t)t * d)[i] = make_uint2(lo, hi);
+      if (y_f32) reinterpret_cast<float4*>(y_f32 + (size_t)t * d)[i] = acc;
+    }
+  }
+}
+
+// out[r, :] = sum_s o[s][r, :] for r < R (split entry point with a K-split down GEMM).
+__global__ void __launch_bounds__(256) reduce_splits_kernel(const float* __restrict__ o, int splits,
+                                                            size_t split_stride,
+                                                            const int32_t* __restrict__ total_rows,
+                                                            int64_t rcap, int d,
+                                                            float* __restrict__ out) {
+  const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
+  const int nv = d / 4;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+      float4 v = reinterpret_cast<const float4*>(o + (size_t)r * d)[i];
+      for (int s = 1; s < splits; ++s) {
+        const float4 u = reinterpret_cast<const float4*>(o + s * split_stride + (size_t)r * d)[i];
+        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+      }
+      reinterpret_cast<float4*>(out + (size_t)r * d)[i] = v;
+    }
+  }
+}
+
+static int row_grid(int64_t rows) {
+  return (int)std::min<int64_t>(std::max<int64_t>(rows, 1), 8LL * num_sms());
+}
+
+cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
+                           const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s) {
+  requant_kernel<<<row_grid(p.Rcap), 256, 0, s>>>(act, amax, total_rows, p.Rcap, p.F, aq, s2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t split_stride,
+                           const float* topk_w, const int32_t* inv_row, const float* shared_src,
+                           const int32_t* shared_row0, int shared_splits, uint16_t* y,
+                           float* y_f32, cudaStream_t s) {
+  // status pointer: the combine of the split entry point has no workspace; pass none
+  combine_kernel<<<row_grid(p.T), 256, 0, s>>>(o, splits, split_stride, topk_w, inv_row, p.k_max,
+                                               p.Rcap, shared_src, shared_row0, shared_splits,
+                                               split_stride, p.T, p.d, y, y_f32, nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_splits(const Plan& p, const float* o, int splits, size_t split_stride,
+                                 const int32_t* total_rows, float* out, cudaStream_t s) {
+  reduce_splits_kernel<<<row_grid(p.Rcap), 256, 0, s>>>(o, splits, split_stride, total_rows,
+                                                        p.Rcap, p.d, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

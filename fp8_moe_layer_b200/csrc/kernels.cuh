@@ -1,0 +1,82 @@
+// Internal launch plan and kernel launchers of the FP8 MoE layer (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kBK = 128;            // bytes (= e4m3 elements) of K per pipeline stage
+constexpr int kRouterTile = 32;     // router logits tile: 32 tokens x 32 experts x 32 of d
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxK = 32;
+
+// Everything the host decides for one (dims) configuration: tile sizes, split counts and the
+// carve-up of the workspace. Offsets are bytes from the workspace base, 256-byte aligned.
+struct Plan {
+  int T, d, E, F, k_max, Fs;
+  bool shared;
+  int G;             // GEMM groups: E routed experts (+1 shared expert)
+  int64_t Rcap;      // routed-row capacity: T*k_max (+T shared rows)
+  int64_t Rpad;      // rows allocated for row-indexed buffers (>= Rcap, >= 256)
+  int BN;            // token tile of the grouped GEMMs (MMA N)
+  int r_splits, r_chunks_per_split;           // router: split of d into 32-wide chunks
+  int g1_kb, g1_m_tiles;                      // gate/up GEMM: K blocks (d/128), 64-row tiles
+  int g2_kb, g2_m_tiles, g2_splits, g2_kb_per_split;  // down GEMM
+  size_t off_status, off_part, off_ids, off_w, off_offsets, off_tiles, off_perm, off_inv;
+  size_t off_xq, off_xs, off_xqp, off_xsp, off_amax, off_act, off_aq, off_s2, off_o;
+  size_t bytes;
+};
+
+// Arguments of one grouped GEMM launch (tile decode + epilogue).
+struct GemmArgs {
+  const int32_t* group_offsets;  // [G+1] first routed row of each group
+  const int32_t* tile_prefix;    // [G+1] prefix sum over groups of ceil(rows / BN)
+  int G, E_routed;               // groups >= E_routed use the shared-expert weights
+  int m_tiles, splits, kb_per_split, num_kb;
+  int M_valid;                   // valid weight rows: F (gate/up halves) or d (down)
+  const float* row_scale;        // [Rpad] activation scale of each routed row
+  const float* w_scale;          // [E, w_scale_ld] per-output-channel weight scales
+  const float* w_scale_shared;   // [w_scale_ld] shared expert (or null)
+  int w_scale_ld;                // 2F (gate/up) or d (down)
+  float* out;                    // gate/up: act [Rpad, F]; down: o [splits][Rpad, d]
+  int out_ld;
+  size_t out_split_stride;       // elements between split partials
+  uint32_t* row_amax;            // gate/up: [Rpad] |act| max as fp32 bits
+  int* status;
+};
+
+int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p);
+
+cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
+                                 float* part, cudaStream_t s);
+cudaError_t launch_topk_quant(const Plan& p, const float* part, const float* bias, int k,
+                              const int32_t* k_per_token, int32_t* ids, float* w,
+                              const uint16_t* hidden, uint8_t* xq, float* xs, bool do_route,
+                              bool do_quant, int* status, cudaStream_t s);
+cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
+                           int* status, cudaStream_t s);
+cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* tiles, int* status,
+                               cudaStream_t s);
+cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, const int32_t* perm,
+                          const int32_t* total_rows, uint8_t* xqp, float* xsp, uint32_t* amax,
+                          int* status, cudaStream_t s);
+cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
+                               const CUtensorMap& acts, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
+                             const CUtensorMap& acts, const GemmArgs& a, cudaStream_t s);
+cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
+                           const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s);
+cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t split_stride,
+                           const float* topk_w, const int32_t* inv_row, const float* shared_src,
+                           const int32_t* shared_row0, int shared_splits, uint16_t* y,
+                           float* y_f32, cudaStream_t s);
+cudaError_t launch_reduce_splits(const Plan& p, const float* o, int splits, size_t split_stride,
+                                 const int32_t* total_rows, float* out, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace moe

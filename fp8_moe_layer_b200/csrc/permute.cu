@@ -1,0 +1,234 @@
+// Grouping of the routed (token, slot) pairs by expert: per-warp histograms, an exclusive prefix
+// sum over experts, and a stable scatter so routed rows are ordered by (expert, token). Then the
+// gather that lays the quantised token rows out in that order for the grouped GEMMs.
+//
+// Method: "Routage MoE entre GPU" (viite.ai) -- only the selected experts process a token; the
+// tokens are dispatched to their experts and their order restored at the combine.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+constexpr int kPermThreads = 1024;
+constexpr int kPermWarps = kPermThreads / 32;
+
+// Exclusive scan of one int per thread over a 1024-thread block; returns the block total too.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int ws = warp_sums[lane];
+    int wincl = ws;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, wincl, off);
+      if (lane >= off) wincl += o;
+    }
+    warp_sums[lane] = wincl - ws;          // exclusive prefix of warp totals
+    if (lane == 31) warp_sums[32] = wincl;
+  }
+  __syncthreads();
+  total = warp_sums[32];
+  const int r = warp_sums[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+// Single block. Warp w owns tokens [w*chunk, (w+1)*chunk) and walks its (token, slot) pairs in
+// token-major order, 32 at a time. Lanes holding the same expert find each other with
+// __match_any_sync; a lane's rank among them plus the warp's running cursor for that expert
+// gives its row, so rows inside an expert are in ascending token order.
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(
+    const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
+    int E, int has_shared, int BN, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv, int32_t* __restrict__ tiles, int* status) {
+  extern __shared__ int hist[];                  // [kPermWarps][E]
+  __shared__ int warp_sums[33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kPermWarps * E; i += kPermThreads) hist[i] = 0;
+  __syncthreads();
+
+  const int chunk = (T + kPermWarps - 1) / kPermWarps;
+  const int t_begin = min(T, warp * chunk), t_end = min(T, t_begin + chunk);
+  const long long i_begin = (long long)t_begin * k_max, i_end = (long long)t_end * k_max;
+  int* my_hist = hist + warp * E;
+
+  // pass 1: per-warp counts
+  for (long long base = i_begin; base < i_end; base += 32) {
+    const long long idx = base + lane;
+    if (idx < i_end) {
+      const int t = (int)(idx / k_max), j = (int)(idx % k_max);
+      const int kt = k_per_token ? k_per_token[t] : k;
+      if (j < kt) {
+        const int e = ids[idx];
+        if (e >= 0 && e < E) atomicAdd(&my_hist[e], 1);
+        else report(status, kStatusDeviceCheck, kWherePermute, t);
+      }
+    }
+  }
+  __syncthreads();
+
+  // pass 2: expert totals, exclusive scan -> offsets, per-warp cursors, GEMM tile prefix
+  int total_rows = 0, total_tiles = 0;
+  {
+    const int e = threadIdx.x;                 // E <= 1024 = blockDim
+    int cnt = 0;
+    if (e < E)
+      for (int w = 0; w < kPermWarps; ++w) cnt += hist[w * E + e];
+    const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
+    if (e < E) {
+      offsets[e] = off;
+      int run = off;
+      for (int w = 0; w < kPermWarps; ++w) {
+        const int c = hist[w * E + e];
+        hist[w * E + e] = run;
+        run += c;
+      }
+    }
+    const int nt = e < E ? (cnt + BN - 1) / BN : 0;
+    const int toff = block_exclusive_scan(nt, warp_sums, total_tiles);
+    if (e < E) tiles[e] = toff;
+    if (threadIdx.x == 0) {
+      offsets[E] = total_rows;
+      if (has_shared) {
+        offsets[E + 1] = total_rows + T;
+        tiles[E] = total_tiles;
+        tiles[E + 1] = total_tiles + (T + BN - 1) / BN;
+      } else {
+        tiles[E] = total_tiles;
+      }
+    }
+  }
+  __syncthreads();
+
+  // pass 3: stable scatter
+  for (long long base = i_begin; base < i_end; base += 32) {
+    const long long idx = base + lane;
+    bool valid = false;
+    int t = 0, e = -1;
+    if (idx < i_end) {
+      t = (int)(idx / k_max);
+      const int j = (int)(idx % k_max);
+      const int kt = k_per_token ? k_per_token[t] : k;
+      if (j < kt) {
+        e = ids[idx];
+        valid = e >= 0 && e < E;
+      }
+      if (!valid) inv[idx] = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : E + lane);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int cursor = valid ? my_hist[e] : 0;
+    __syncwarp();
+    if (valid) {
+      const int r = cursor + rank;
+      perm[r] = t;
+      inv[idx] = r;
+      if (rank == 0) my_hist[e] = cursor + __popc(peers);
+    }
+    __syncwarp();
+  }
+  if (has_shared)
+    for (int t = threadIdx.x; t < T; t += kPermThreads) perm[total_rows + t] = t;
+}
+
+// For caller-provided offsets (split entry point): validate and build the GEMM tile prefix.
+__global__ void __launch_bounds__(kPermThreads) tile_prefix_kernel(
+    const int32_t* __restrict__ offsets, int E, int64_t rcap, int BN, int32_t* __restrict__ tiles,
+    int* status) {
+  __shared__ int warp_sums[33];
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  const int e = threadIdx.x;
+  int nt = 0;
+  if (e < E) {
+    const int a = offsets[e], b = offsets[e + 1];
+    if (a < 0 || b < a || b > rcap) bad = 1;
+    else nt = (b - a + BN - 1) / BN;
+  }
+  int total = 0;
+  const int toff = block_exclusive_scan(nt, warp_sums, total);
+  __syncthreads();
+  if (bad) {
+    // inconsistent offsets: publish an empty tile list so no GEMM work is done
+    if (e <= E) tiles[e] = 0;
+    if (threadIdx.x == 0) report(status, kStatusDeviceCheck, kWhereTilePrefix, 0);
+    return;
+  }
+  if (e < E) tiles[e] = toff;
+  if (threadIdx.x == 0) tiles[E] = total;
+}
+
+// One warp per routed row: xqp[r, :] = xq[perm[r], :], xsp[r] = xs[perm[r]], amax[r] = 0.
+// A token index outside [0, T) (caller-provided permutation) gives a zero row and flags
+// MOE_ERR_DEVICE_CHECK.
+__global__ void __launch_bounds__(256) gather_rows_kernel(
+    const uint8_t* __restrict__ xq, const float* __restrict__ xs, const int32_t* __restrict__ perm,
+    const int32_t* __restrict__ total_rows, int64_t rcap, int T, int d, uint8_t* __restrict__ xqp,
+    float* __restrict__ xsp, uint32_t* __restrict__ amax, int* status) {
+  const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
+  const int lane = threadIdx.x & 31;
+  const int nv = d / 16;
+  for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < R; r += gridDim.x * 8) {
+    const int t = perm[r];
+    const bool ok = t >= 0 && t < T;
+    uint4* dst = reinterpret_cast<uint4*>(xqp + (size_t)r * d);
+    if (ok) {
+      const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
+      for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+    } else {
+      for (int i = lane; i < nv; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (lane == 0) {
+      xsp[r] = ok ? xs[t] : 0.f;
+      amax[r] = 0u;
+      if (!ok) report(status, kStatusDeviceCheck, kWhereGather, r);
+    }
+  }
+}
+
+cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
+                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
+                           int* status, cudaStream_t s) {
+  const size_t smem = sizeof(int) * kPermWarps * p.E;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPermWarps * kMaxExperts * (int)sizeof(int));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  permute_kernel<<<1, kPermThreads, smem, s>>>(ids, p.T, p.k_max, k, k_per_token, p.E,
+                                               p.shared ? 1 : 0, p.BN, offsets, perm, inv, tiles,
+                                               status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* tiles, int* status,
+                               cudaStream_t s) {
+  tile_prefix_kernel<<<1, kPermThreads, 0, s>>>(offsets, p.E, (int64_t)p.T * p.k_max, p.BN, tiles,
+                                                status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, const int32_t* perm,
+                          const int32_t* total_rows, uint8_t* xqp, float* xsp, uint32_t* amax,
+                          int* status, cudaStream_t s) {
+  const int64_t blocks_needed = (p.Rcap + 7) / 8;
+  const int grid = (int)std::min<int64_t>(std::max<int64_t>(blocks_needed, 1), 8LL * num_sms());
+  gather_rows_kernel<<<grid, 256, 0, s>>>(xq, xs, perm, total_rows, p.Rcap, p.T, p.d, xqp, xsp,
+                                          amax, status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
