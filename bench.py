@@ -51,8 +51,8 @@ def parse_args():
 
 
 def dist_env():
-    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
-            int(os.environ.get("LOCAL_RANK", 0)))
+    from fp8_moe_layer_b200.replicas import rank_env
+    return rank_env()
 
 
 def peaks():
@@ -228,7 +228,8 @@ def run_ours(args):
     from fp8_moe_layer_b200 import ops
 
     shape = I.WORKLOADS[args.workload]
-    inp = I.make_inputs(shape, seed=rank, quant_device=f"cuda:{local}")
+    from fp8_moe_layer_b200 import replicas
+    inp = I.make_inputs(shape, seed=replicas.replica_seed(0, rank), quant_device=f"cuda:{local}")
     layer = ops.MoELayerFP8(inp, device=f"cuda:{local}")
     dev = torch.device(f"cuda:{local}")
     hidden = inp.hidden.to(dev)
@@ -284,10 +285,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     e2e_ms = float(np.mean([e_start[i].elapsed_time(e_end[i]) for i in range(args.steps)]))
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = replicas.max_over_ranks([ms, e2e_ms], device=dev)
     total_tokens = shape.T * world
     if rank != 0:
         if world > 1:
@@ -307,7 +305,7 @@ def run_ours(args):
                    sample=f"{n} of {shape.T} tokens through the FFN and combine; routing and "
                           f"grouping of all {shape.T} tokens ({dt:.1f} s)")
     line = dict(
-        metric=METRIC, value=total_tokens / (ms * 1e-3), unit="tokens/s", n_gpus=world,
+        metric=METRIC, value=replicas.aggregate_tokens_per_s(shape.T, world, ms), unit="tokens/s", n_gpus=world,
         steps=args.steps, warmup=args.warmup, ms_per_step=ms, us_per_layer=ms * 1e3,
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="fp8_e4m3",
         data="synthetic (seeded, random-init weights of the layer shape)",
@@ -324,7 +322,7 @@ def run_ours(args):
                             active_experts=work["active_experts"],
                             routed_rows=work["routed_rows"], flops=work["flops"]),
         stage_us=stages,
-        e2e=dict(value=total_tokens / (e2e_ms * 1e-3), unit="tokens/s",
+        e2e=dict(value=replicas.aggregate_tokens_per_s(shape.T, world, e2e_ms), unit="tokens/s",
                  h2d_bytes_per_step=shape.T * shape.d * 2, d2h_bytes_per_step=shape.T * shape.d * 2),
         gpu_launches=ops.NUM_STAGES * args.steps,
         clocks=clocks.summary(),

@@ -235,6 +235,9 @@ def moe_forward(hidden, router_w, router_bias, k, k_per_token, w13, w13_scale, w
                        inv_row=torch.empty(T, k_max, dtype=torch.int32, device=dev),
                        y_f32=torch.empty(T, d, dtype=torch.float32, device=dev))
         if stage_events is not None:
+            for e in stage_events:            # torch creates its events lazily, on first record
+                if e is not None and not e.cuda_event:
+                    e.record()
             ev_arr = (ctypes.c_void_p * (NUM_STAGES + 1))(
                 *[ctypes.c_void_p(e.cuda_event if e is not None else 0) for e in stage_events])
         dbg_struct = MoEDebugOut(*(dbg[n].data_ptr() if n in dbg else None for n in

@@ -62,27 +62,50 @@ def bf16_half_ulp(v: np.ndarray) -> np.ndarray:
     return np.ldexp(1.0, np.maximum(x - 1, -126) - 8)
 
 
+def order_tie_tokens(logits: np.ndarray, k_t: np.ndarray, gap: float = NEAR_TIE) -> np.ndarray:
+    """Tokens with two of their k_t selected logits within ``gap`` of each other: the slot order
+    of those two experts is not decided by fp32 vs float64 evaluation."""
+    s = -np.sort(-logits, axis=-1)
+    out = []
+    for t in range(logits.shape[0]):
+        kk = int(k_t[t])
+        if kk > 1 and np.min(s[t, :kk - 1] - s[t, 1:kk]) < gap:
+            out.append(t)
+    return np.asarray(out, dtype=np.int64)
+
+
 def check_routing(gpu_ids: np.ndarray, gpu_w: np.ndarray, ref: dict):
-    """Bit-exact ids on every token without a near tie at its k-th place; on near-tie tokens the
-    GPU's choice must be a valid top-k (every chosen logit within NEAR_TIE of the k-th best).
-    Returns the number of near-tie tokens and how many of them differed."""
+    """Routing parity.
+    * Tokens without any near tie: ids bit-exact (set and slot order), weights within WEIGHT_ATOL.
+    * Near tie at the k-th place (k-th and (k+1)-th oracle logits within NEAR_TIE): the GPU's
+      choice must be a valid top-k -- k_t distinct experts, each within NEAR_TIE of the k-th.
+    * Near tie inside the selection only: the SET is bit-exact, the GPU order is descending in
+      the oracle logits up to NEAR_TIE, and each expert's weight matches.
+    Returns (boundary near ties, how many of them chose differently, order-only near ties)."""
     logits, ids, w, k_t = ref["logits"], ref["topk_ids"], ref["topk_w"], ref["k_t"]
     near = set(O.near_tie_tokens(logits, k_t, NEAR_TIE).tolist())
+    order = set(order_tie_tokens(logits, k_t, NEAR_TIE).tolist()) - near
     differed = 0
     for t in range(ids.shape[0]):
         kt = int(k_t[t])
         assert np.all(gpu_ids[t, kt:] == -1) and np.all(gpu_w[t, kt:] == 0), t
+        sel = gpu_ids[t, :kt]
         if t in near:
-            if not np.array_equal(gpu_ids[t, :kt], ids[t, :kt]):
+            if not np.array_equal(sel, ids[t, :kt]):
                 differed += 1
                 kth = np.sort(logits[t])[::-1][kt - 1]
-                sel = gpu_ids[t, :kt]
                 assert len(set(sel.tolist())) == kt
                 assert np.all(logits[t, sel] >= kth - NEAR_TIE), t
             continue
-        assert np.array_equal(gpu_ids[t, :kt], ids[t, :kt]), (t, gpu_ids[t], ids[t])
+        if t in order:
+            assert set(sel.tolist()) == set(ids[t, :kt].tolist()), t
+            assert np.all(np.diff(logits[t, sel]) <= NEAR_TIE), t
+            ref_w = dict(zip(ids[t, :kt].tolist(), w[t, :kt].tolist()))
+            assert max(abs(gpu_w[t, j] - ref_w[int(e)]) for j, e in enumerate(sel)) <= WEIGHT_ATOL
+            continue
+        assert np.array_equal(sel, ids[t, :kt]), (t, gpu_ids[t], ids[t])
         assert np.abs(gpu_w[t, :kt] - w[t, :kt]).max() <= WEIGHT_ATOL, (t, gpu_w[t], w[t])
-    return len(near), differed
+    return len(near), differed, len(order)
 
 
 def check_grouping(gpu_offsets, gpu_perm, gpu_inv, ids, k_t, E):

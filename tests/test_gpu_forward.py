@@ -35,7 +35,7 @@ def forward_and_check(ops, inp, sample=None, seed=0):
     k_t = O.token_k(s.T, s.k, H.np_(inp.k_per_token))
     ids = O.select_topk(logits, k_t, s.k_max)
     route_ref = dict(logits=logits, topk_ids=ids, topk_w=O.routing_weights(logits, ids), k_t=k_t)
-    n_near, differed = H.check_routing(gpu["topk_ids"], gpu["topk_w"], route_ref)
+    n_near, differed, n_order = H.check_routing(gpu["topk_ids"], gpu["topk_w"], route_ref)
     H.check_grouping(gpu["expert_offsets"], gpu["perm_token"], gpu["inv_row"],
                      gpu["topk_ids"], k_t, s.E)
 
@@ -48,7 +48,7 @@ def forward_and_check(ops, inp, sample=None, seed=0):
     ref = H.run_oracle(inp, tokens=tokens)
     stats = H.check_output(y[tokens], torch.from_numpy(gpu["y_f32"][tokens]), ref["y64"], s.name)
     print(f"{s.name}: tokens checked {len(tokens)}/{s.T}, near ties {n_near} "
-          f"(differing {differed}), {stats}")
+          f"(differing {differed}), order-only ties {n_order}, {stats}")
     return y, dbg, stats
 
 
