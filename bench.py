@@ -4,11 +4,13 @@ A step is one pass of the whole layer (router, top-k, quantisation, permutation,
 FFN, combine) over one batch of synthetic tokens of the Mixtral-8x7B-shaped workload
 (d=4096, E=8, F=14336, top-2, T=512 tokens per GPU) through the C ABI entry point moe_forward.
 
-* value: tokens/s over all ranks, device time (CUDA events on the launching stream) with every
-  input resident in HBM; L2 flushed (256 MiB write) between steps, outside the timed events.
+* value: tokens/s over all ranks, device time (CUDA events on the launching stream around each
+  step) with every input resident in HBM; L2 flushed (256 MiB write + 256 MiB read) between
+  steps, outside the timed events.
 * e2e: the same metric with the step's hidden states copied from pinned host memory and the
   output copied back inside the timed region.
-* roofline: the dominant kernel (the gate/up GEMM + SwiGLU) timed by events around its launch.
+* roofline: the dominant kernel (the gate/up GEMM + SwiGLU) timed by events around its launch,
+  in a second pass over the same steps with an event before every kernel of the layer.
 * cpu_baseline (rank 0, N=1): the CPU oracle timed on a bounded token sample.
 * --impl reference: the CPU oracle as the reference arm (no GPU work).
 Multi-GPU: independent replicas (one batch per rank, seed = rank), no collective on the path.
@@ -173,6 +175,20 @@ def cpu_oracle_time(inp, n_tokens: int, seed: int = 0):
     return len(tokens), dt
 
 
+def launches_per_step(shape) -> int:
+    """Kernels one moe_forward launches for this shape (the library's router and grouping paths:
+    fused router for E <= 32, tensor-core router (split + GEMM + top-k) for E > 32 and T >= 64,
+    else CUDA-core logits + top-k; one grouping kernel for T*k_max <= 8192, else three)."""
+    if shape.E <= 32 and shape.d <= 8192:
+        router = 1
+    elif shape.T >= 64:
+        router = 3
+    else:
+        router = 2
+    permute = 1 if shape.T * shape.k_max <= 8192 else 3
+    return router + permute + 5      # gather, gate/up GEMM, requant, down GEMM, combine
+
+
 def host_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -235,7 +251,10 @@ def run_ours(args):
     hidden = inp.hidden.to(dev)
     kpt = None if inp.k_per_token is None else inp.k_per_token.to(dev)
     y = torch.empty(shape.T, shape.d, dtype=torch.bfloat16, device=dev)
+    # L2 flush between timed steps: write one buffer larger than L2, then read another, so the
+    # next step starts with a cold L2 that holds no dirty lines
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -246,23 +265,38 @@ def run_ours(args):
     _, dbg = layer(hidden, kpt, debug=True)
     work = algorithmic(shape, dbg["expert_offsets"].cpu().numpy())
 
-    n_ev = ops.NUM_STAGES + 1
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-              for _ in range(args.steps)]
+    # (a) the step time: events around each moe_forward only (no events between its kernels,
+    #     which would serialise the programmatic launches)
+    s_start = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    s_end = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)                       # evict L2 (outside the timed events)
-            layer(hidden, kpt, y=y, stage_events=events[i])
+            flush_rd.sum()
+            s_start[i].record(stream)
+            layer(hidden, kpt, y=y)
+            s_end[i].record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    step_ms = np.array([s_start[i].elapsed_time(s_end[i]) for i in range(args.steps)])
+    ms = float(step_ms.mean())
+
+    # (b) per-kernel times: the same steps with an event before every kernel of the layer
+    n_ev = ops.NUM_STAGES + 1
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+              for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        flush_rd.sum()
+        layer(hidden, kpt, y=y, stage_events=events[i])
+    torch.cuda.synchronize(dev)
     stage_ms = np.array([[events[i][j].elapsed_time(events[i][j + 1]) for j in range(n_ev - 1)]
                          for i in range(args.steps)])
-    step_ms = np.array([events[i][0].elapsed_time(events[i][-1]) for i in range(args.steps)])
-    ms = float(step_ms.mean())
 
     # e2e: pinned host hidden -> device, layer, y -> pinned host, all inside the events
     h_host = inp.hidden.pin_memory()
@@ -277,6 +311,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
+        flush_rd.sum()
         e_start[i].record(stream)
         h_dev.copy_(h_host, non_blocking=True)
         layer(h_dev, kpt, y=y)
@@ -311,7 +346,7 @@ def run_ours(args):
         data="synthetic (seeded, random-init weights of the layer shape)",
         config=dict(workload=args.workload, T=shape.T, d=shape.d, E=shape.E, F=shape.F,
                     k=shape.k, F_shared=shape.F_shared, parallelism=f"replicas x{world}",
-                    l2="flushed between timed steps (256 MiB write outside the events)"),
+                    l2="flushed between timed steps (256 MiB write + 256 MiB read, outside the events)"),
         roofline=dict(bound="hbm", kernel="gemm_gateup_swiglu", achieved=g1_gbs,
                       peak=pk["hbm_gbs"], unit="GB/s", frac=g1_gbs / pk["hbm_gbs"],
                       traffic=ncu_traffic(f"gemm_gateup_{args.workload}"),
@@ -324,7 +359,7 @@ def run_ours(args):
         stage_us=stages,
         e2e=dict(value=replicas.aggregate_tokens_per_s(shape.T, world, e2e_ms), unit="tokens/s",
                  h2d_bytes_per_step=shape.T * shape.d * 2, d2h_bytes_per_step=shape.T * shape.d * 2),
-        gpu_launches=ops.NUM_STAGES * args.steps,
+        gpu_launches=launches_per_step(shape) * args.steps,
         clocks=clocks.summary(),
         cpu_baseline=cpu,
     )

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
                                                       int64_t rcap, int F,
                                                       uint8_t* __restrict__ aq,
                                                       float* __restrict__ s2) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
   const int nv = F / 4;
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
@@ -44,6 +46,8 @@ __global__ void __launch_bounds__(256) combine_kernel(
     const float* __restrict__ shared_src, const int32_t* __restrict__ shared_row0,
     int shared_splits, size_t shared_split_stride, int T, int d, uint16_t* __restrict__ y,
     float* __restrict__ y_f32, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   __shared__ int rows[kMaxK];
   __shared__ float wts[kMaxK];
   const int nv = d / 4;
@@ -99,6 +103,8 @@ __global__ void __launch_bounds__(256) reduce_splits_kernel(const float* __restr
                                                             const int32_t* __restrict__ total_rows,
                                                             int64_t rcap, int d,
                                                             float* __restrict__ out) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
   const int nv = d / 4;
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
@@ -119,7 +125,7 @@ static int row_grid(int64_t rows) {
 
 cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
                            const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s) {
-  requant_kernel<<<row_grid(p.Rcap), 256, 0, s>>>(act, amax, total_rows, p.Rcap, p.F, aq, s2);
+  launch_pdl(requant_kernel, dim3(row_grid(p.Rcap)), dim3(256), 0, s, act, amax, total_rows, p.Rcap, p.F, aq, s2);
   return cudaGetLastError();
 }
 
@@ -128,7 +134,7 @@ cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t spl
                            const int32_t* shared_row0, int shared_splits, uint16_t* y,
                            float* y_f32, cudaStream_t s) {
   // status pointer: the combine of the split entry point has no workspace; pass none
-  combine_kernel<<<row_grid(p.T), 256, 0, s>>>(o, splits, split_stride, topk_w, inv_row, p.k_max,
+  launch_pdl(combine_kernel, dim3(row_grid(p.T)), dim3(256), 0, s, o, splits, split_stride, topk_w, inv_row, p.k_max,
                                                p.Rcap, shared_src, shared_row0, shared_splits,
                                                split_stride, p.T, p.d, y, y_f32, nullptr);
   return cudaGetLastError();
@@ -136,7 +142,7 @@ cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t spl
 
 cudaError_t launch_reduce_splits(const Plan& p, const float* o, int splits, size_t split_stride,
                                  const int32_t* total_rows, float* out, cudaStream_t s) {
-  reduce_splits_kernel<<<row_grid(p.Rcap), 256, 0, s>>>(o, splits, split_stride, total_rows,
+  launch_pdl(reduce_splits_kernel, dim3(row_grid(p.Rcap)), dim3(256), 0, s, o, splits, split_stride, total_rows,
                                                         p.Rcap, p.d, out);
   return cudaGetLastError();
 }

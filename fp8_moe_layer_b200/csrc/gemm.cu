@@ -10,13 +10,16 @@
 // megakernel" (expert compute on 8-bit weights and activations, intermediates kept on chip).
 //
 // Shape of the work: "swap-AB". The MMA's M = 128 rows come from the WEIGHTS (output channels of
-// one expert) and its N = BN columns from the routed TOKEN rows of that expert, so a decode
-// batch with a handful of tokens per expert still fills the 128-row tensor-core tile and every
-// weight byte is streamed from HBM once. A gate/up tile holds 64 gate rows and the matching 64
-// up rows (two TMA boxes), so SwiGLU is computed inside one CTA.
+// one expert) and its N columns from the routed TOKEN rows of that expert, so a decode batch with
+// a handful of tokens per expert still fills the 128-row tensor-core tile and every weight byte
+// is streamed from HBM once. A tile loads and multiplies only its valid token rows (N = rows
+// rounded up to 16, chosen per tile at run time). A gate/up tile holds 64 gate rows and the
+// matching 64 up rows (two TMA boxes), so SwiGLU is computed inside one CTA.
 //
-// Persistent kernel, one CTA per SM, static round-robin over tiles (group, m-tile, K-split,
-// n-tile) with n fastest so CTAs working on the same weight tile at the same time share it in L2.
+// Pipeline: a ring of shared-memory stages, each holding one K-block of weights (16 KB) and of the
+// tile's token rows; as many stages as fit in 227 KB. Persistent kernel, one CTA per SM, static
+// round-robin over tiles (group, m-tile, K-split, n-tile) with n fastest so CTAs working on the
+// same weight tile at the same time share it in L2.
 // Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = TMEM allocator, warps 4-7 =
 // epilogue (warp w reads TMEM lanes 32*(w%4) .. +31). Two TMEM accumulator buffers let the
 // epilogue of one tile overlap the main loop of the next. Every wait is bounded (about 1 s); on
@@ -42,10 +45,13 @@ struct GemmCfg {
   static constexpr int STAGES_FIT = (SMEM_MAX - 1024 - XCHG_BYTES - BAR_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCHG_BYTES + BAR_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;   // two accumulator buffers
+  // two accumulator buffers; the allocation is a power of two >= 32 columns
+  static constexpr int TMEM_COLS = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128
+                                   : 2 * BN <= 256 ? 256 : 512;
   static constexpr int CW = BN < 32 ? BN : 32;                 // epilogue column chunk
   static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128");
+  static_assert(BN % CW == 0, "epilogue chunks");
 };
 
 // tile -> (group g, m-tile, K-split s, n-tile). Group g covers tiles
@@ -69,11 +75,27 @@ __device__ __forceinline__ void decode_tile(const GemmArgs& a, int tile, int& g,
   m = rest / a.splits;
 }
 
+// Valid token rows of the tile starting at row0 of group g, rounded up to a multiple of 16.
+template <int BN>
+__device__ __forceinline__ int tile_rows16(const GemmArgs& a, int g, int row0) {
+  const int rows = min(BN, a.group_offsets[g + 1] - row0);
+  return (rows + 15) & ~15;
+}
+
+// silu(g) = g / (1 + e^-g) with the fast exponential and division; the exponent is clamped so the
+// denominator stays finite (silu(g) < 1e-30 in magnitude below g = -80).
+__device__ __forceinline__ float silu(float g) {
+  return __fdividef(g, 1.f + __expf(fminf(-g, 80.f)));
+}
+
 template <int BN, bool GATEUP>
 __global__ void __launch_bounds__(256, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_a_shared,
-                        const __grid_constant__ CUtensorMap map_b, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap map_b64,
+                        const __grid_constant__ CUtensorMap map_b16, const GemmArgs args) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   using C = GemmCfg<BN, GATEUP>;
   constexpr int kWhere = GATEUP ? kWhereGemm1 : kWhereGemm2;
   extern __shared__ uint8_t smem_raw[];
@@ -117,7 +139,8 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       tma_prefetch_map(&map_a);
       tma_prefetch_map(&map_a_shared);
-      tma_prefetch_map(&map_b);
+      tma_prefetch_map(&map_b64);
+      tma_prefetch_map(&map_b16);
       const uint64_t pol_w = l2_policy_evict_first();   // weights: streamed once
       const uint64_t pol_x = l2_policy_evict_last();    // activations: reused by every m-tile
       int stage = 0, issued = 0;
@@ -127,6 +150,8 @@ __global__ void __launch_bounds__(256, 1)
         int g, m, n, s;
         decode_tile(args, tile, g, m, n, s);
         const int row0 = args.group_offsets[g] + n * BN;
+        const int rows16 = tile_rows16<BN>(args, g, row0);   // valid token rows, rounded to 16
+        const uint32_t stage_bytes = C::A_BYTES + rows16 * kBK;
         const int kb0 = s * args.kb_per_split;
         const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
         const bool sh = g >= args.E_routed;
@@ -139,14 +164,21 @@ __global__ void __launch_bounds__(256, 1)
             break;
           }
           uint8_t* sa = stages + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          mbar_arrive_expect_tx(&full[stage], stage_bytes);
           if (GATEUP) {
             tma_load_4d(sa, ma, &full[stage], kb * kBK, m * 64, 0, ga, pol_w);
             tma_load_4d(sa + C::A_BYTES / 2, ma, &full[stage], kb * kBK, m * 64, 1, ga, pol_w);
           } else {
             tma_load_3d(sa, ma, &full[stage], kb * kBK, m * 128, ga, pol_w);
           }
-          tma_load_2d(sa + C::A_BYTES, &map_b, &full[stage], kb * kBK, row0, pol_x);
+          // only the tile's valid token rows: 64-row boxes, then 16-row boxes
+          uint8_t* sb = sa + C::A_BYTES;
+          int r = 0;
+          if constexpr (BN >= 64)
+            for (; r + 64 <= rows16; r += 64)
+              tma_load_2d(sb + r * kBK, &map_b64, &full[stage], kb * kBK, row0 + r, pol_x);
+          for (; r < rows16; r += 16)
+            tma_load_2d(sb + r * kBK, &map_b16, &full[stage], kb * kBK, row0 + r, pol_x);
           ++issued;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -169,7 +201,6 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (one thread)
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(128, BN);
       int stage = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -178,6 +209,9 @@ __global__ void __launch_bounds__(256, 1)
         decode_tile(args, tile, g, m, n, s);
         const int kb0 = s * args.kb_per_split;
         const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
+        // MMA N = the tile's valid rows rounded up to 16 (M = 128 takes N = 16 .. 256 by 16)
+        const uint32_t idesc =
+            idesc_e4m3_f32(128, tile_rows16<BN>(args, g, args.group_offsets[g] + n * BN));
         const int ab = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[ab], aph ^ 1u)) {
@@ -217,7 +251,6 @@ __global__ void __launch_bounds__(256, 1)
     // After a timeout a warp keeps walking the tile list and joins every named barrier (so the
     // other epilogue warps never wait on it) but touches neither TMEM nor global memory.
     const int q = warp & 3;
-    const int tid_e = threadIdx.x - 128;
     bool bad = false;
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
@@ -228,7 +261,7 @@ __global__ void __launch_bounds__(256, 1)
       if (!bad) {
         const bool ok = mbar_wait(&tfull[ab], aph);
         bad = __any_sync(0xffffffffu, !ok);         // warp-uniform: TMEM loads are .sync.aligned
-        if (bad && lane == 0) report(args.status, kStatusDeviceTimeout, kWhere, 4);
+        if (bad && lane == 0) report(args.status, kStatusDeviceTimeout, kWhere, 5);
       }
       tc_fence_after_sync();
       const int row0 = args.group_offsets[g] + n * BN;
@@ -237,13 +270,14 @@ __global__ void __launch_bounds__(256, 1)
       const float* wsc = sh ? args.w_scale_shared : args.w_scale + (size_t)g * args.w_scale_ld;
       const uint32_t tbase = tmem_base + ab * BN + (static_cast<uint32_t>(32 * q) << 16);
       if constexpr (GATEUP) {
+        // TMEM lane 32q+i holds gate row (q<2) or up row (q>=2) 32*(q&1)+i of this 64-row half
+        // pair. Step 1: every warp parks its rows (scaled by the weight scale) in smem.
+        // Step 2: thread (q, lane) takes token column `lane` and the 16 features 16q .. 16q+15:
+        // SwiGLU, one 64-byte store, and the in-thread max |act| for the row amax.
         constexpr int CW = C::CW;
-        const int jj = 32 * (q & 1) + lane;           // row inside the 64-row half
-        const int half = q >> 1;                       // 0: gate rows, 1: up rows
-        const int frow = m * 64 + jj;
-        const float wsv = frow < args.M_valid ? wsc[half * args.M_valid + frow] : 0.f;
-        const int j = tid_e & 63;                      // compute mapping: fixed row j per thread
-        const int f = m * 64 + j;
+        const int frow = m * 64 + 32 * (q & 1) + lane;
+        const float wsv = frow < args.M_valid ? wsc[(q >> 1) * args.M_valid + frow] : 0.f;
+        const int f0 = m * 64 + 16 * q;                // this thread's first feature
         for (int c0 = 0; c0 < nvalid; c0 += CW) {
           if (!bad) {
             uint32_t r[CW];
@@ -256,26 +290,24 @@ __global__ void __launch_bounds__(256, 1)
             for (int c = 0; c < CW; ++c) xr[c] = __uint_as_float(r[c]) * wsv;
           }
           named_bar_sync(1, 128);
-          if (!bad) {
-#pragma unroll 4
-            for (int ii = 0; ii < CW / 2; ++ii) {
-              const int c = (tid_e >> 6) + 2 * ii;      // warp-uniform column
-              const int nn = c0 + c;
-              float act = 0.f;
-              if (nn < nvalid && f < args.M_valid) {
-                const float rs = args.row_scale[row0 + nn];
-                const float gv = xchg[j * C::XCHG_LD + c] * rs;
-                const float uv = xchg[(64 + j) * C::XCHG_LD + c] * rs;
-                act = gv / (1.f + expf(-gv)) * uv;
-                args.out[(size_t)(row0 + nn) * args.out_ld + f] = act;
-              }
-              float a = fabsf(act);
+          const int nn = c0 + lane;
+          if (!bad && lane < CW && nn < nvalid && f0 < args.M_valid) {
+            const float rs = args.row_scale[row0 + nn];
+            float act[16];
+            float amax = 0.f;
 #pragma unroll
-              for (int off = 16; off > 0; off >>= 1)
-                a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
-              if (lane == 0 && nn < nvalid)
-                atomicMax(&args.row_amax[row0 + nn], __float_as_uint(a));
+            for (int jj = 0; jj < 16; ++jj) {
+              const int j = 16 * q + jj;
+              const float gv = xchg[j * C::XCHG_LD + lane] * rs;
+              const float uv = xchg[(64 + j) * C::XCHG_LD + lane] * rs;
+              act[jj] = silu(gv) * uv;
+              amax = fmaxf(amax, fabsf(act[jj]));
             }
+            float4* dst = reinterpret_cast<float4*>(args.out + (size_t)(row0 + nn) * args.out_ld + f0);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_float4(act[4 * v], act[4 * v + 1], act[4 * v + 2], act[4 * v + 3]);
+            atomicMax(&args.row_amax[row0 + nn], __float_as_uint(amax));
           }
           named_bar_sync(1, 128);
         }
@@ -312,8 +344,8 @@ __global__ void __launch_bounds__(256, 1)
 
 namespace {
 template <int BN, bool GATEUP>
-cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& ash, const CUtensorMap& b,
-                          const GemmArgs& args, cudaStream_t s) {
+cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& ash, const CUtensorMap& b64,
+                          const CUtensorMap& b16, const GemmArgs& args, cudaStream_t s) {
   using C = GemmCfg<BN, GATEUP>;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -325,32 +357,36 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& ash, const CU
     if (err != cudaSuccess) return err;
     attr_done[dev] = true;
   }
-  grouped_gemm_kernel<BN, GATEUP><<<num_sms(), 256, C::SMEM, s>>>(a, ash, b, args);
+  launch_pdl(grouped_gemm_kernel<BN, GATEUP>, dim3(num_sms()), dim3(256), C::SMEM, s, a, ash, b64, b16, args);
   return cudaGetLastError();
 }
 
 template <bool GATEUP>
 cudaError_t launch_by_bn(int BN, const CUtensorMap& a, const CUtensorMap& ash,
-                         const CUtensorMap& b, const GemmArgs& args, cudaStream_t s) {
+                         const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& args,
+                         cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_gemm_t<16, GATEUP>(a, ash, b, args, s);
-    case 32: return launch_gemm_t<32, GATEUP>(a, ash, b, args, s);
-    case 64: return launch_gemm_t<64, GATEUP>(a, ash, b, args, s);
-    case 128: return launch_gemm_t<128, GATEUP>(a, ash, b, args, s);
-    case 256: return launch_gemm_t<256, GATEUP>(a, ash, b, args, s);
+    case 16: return launch_gemm_t<16, GATEUP>(a, ash, b64, b16, args, s);
+    case 32: return launch_gemm_t<32, GATEUP>(a, ash, b64, b16, args, s);
+    case 64: return launch_gemm_t<64, GATEUP>(a, ash, b64, b16, args, s);
+    case 128: return launch_gemm_t<128, GATEUP>(a, ash, b64, b16, args, s);
+    case 192: return launch_gemm_t<192, GATEUP>(a, ash, b64, b16, args, s);
+    case 256: return launch_gemm_t<256, GATEUP>(a, ash, b64, b16, args, s);
     default: return cudaErrorInvalidValue;
   }
 }
 }  // namespace
 
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
-                               const CUtensorMap& acts, const GemmArgs& a, cudaStream_t s) {
-  return launch_by_bn<true>(p.BN, w13, w13s, acts, a, s);
+                               const CUtensorMap& acts64, const CUtensorMap& acts16,
+                               const GemmArgs& a, cudaStream_t s) {
+  return launch_by_bn<true>(p.BN, w13, w13s, acts64, acts16, a, s);
 }
 
 cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
-                             const CUtensorMap& acts, const GemmArgs& a, cudaStream_t s) {
-  return launch_by_bn<false>(p.BN, w2, w2s, acts, a, s);
+                             const CUtensorMap& acts64, const CUtensorMap& acts16,
+                             const GemmArgs& a, cudaStream_t s) {
+  return launch_by_bn<false>(p.BN, w2, w2s, acts64, acts16, a, s);
 }
 
 }  // namespace moe

@@ -21,12 +21,12 @@ struct Plan {
   int G;             // GEMM groups: E routed experts (+1 shared expert)
   int64_t Rcap;      // routed-row capacity: T*k_max (+T shared rows)
   int64_t Rpad;      // rows allocated for row-indexed buffers (>= Rcap, >= 256)
-  int BN;            // token tile of the grouped GEMMs (MMA N)
+  int BN;            // token tile of the grouped GEMMs (max MMA N; a tile uses its valid rows)
   int r_splits, r_chunks_per_split;           // router: split of d into 32-wide chunks
   int g1_kb, g1_m_tiles;                      // gate/up GEMM: K blocks (d/128), 64-row tiles
   int g2_kb, g2_m_tiles, g2_splits, g2_kb_per_split;  // down GEMM
-  size_t off_status, off_part, off_ids, off_w, off_offsets, off_tiles, off_perm, off_inv;
-  size_t off_xq, off_xs, off_xqp, off_xsp, off_amax, off_act, off_aq, off_s2, off_o;
+  size_t off_status, off_part, off_ids, off_w, off_offsets, off_tiles, off_perm, off_inv, off_pscr;
+  size_t off_xq, off_xs, off_xqp, off_xsp, off_amax, off_act, off_aq, off_s2, off_o, off_planes;
   size_t bytes;
 };
 
@@ -55,19 +55,40 @@ cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const fl
 cudaError_t launch_topk_quant(const Plan& p, const float* part, const float* bias, int k,
                               const int32_t* k_per_token, int32_t* ids, float* w,
                               const uint16_t* hidden, uint8_t* xq, float* xs, bool do_route,
-                              bool do_quant, int* status, cudaStream_t s);
+                              bool do_quant, const float* refine_w, int* status, cudaStream_t s);
+// Router paths. E <= 32: one fused kernel (logits, top-k, weights, quantisation). E > 32 and
+// T >= 64: tensor-core logits (bf16 split of the fp32 weights) + topk_quant. Otherwise: CUDA-core
+// logits + topk_quant.
+// (the fused router holds a token's row in registers: d <= 8192)
+inline bool router_is_fused(int E, int d) { return E <= 32 && d <= 8192; }
+inline bool router_uses_mma(int E, int T) { return E > 32 && T >= 64; }
+inline bool router_is_fused(const Plan& p) { return router_is_fused(p.E, p.d); }
+inline bool router_uses_mma(const Plan& p) { return router_uses_mma(p.E, p.T); }
+// planes: 3 * E * d bf16 (workspace); map_w over planes [3][E][d], map_x over hidden [T][d]
+cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
+                              const CUtensorMap& map_w, const CUtensorMap& map_x, float* logits,
+                              int* status, cudaStream_t s);
+cudaError_t launch_route_fused(const Plan& p, const uint16_t* hidden, const float* router_w,
+                               const float* bias, int k, const int32_t* k_per_token,
+                               int32_t* ids, float* w, uint8_t* xq, float* xs, bool do_quant,
+                               int* status, cudaStream_t s);
+// scratch: 2 * permute_blocks(p) * E int32 (per-block counts and bases; unused for one block)
+int permute_blocks(const Plan& p);
 cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
-                           int* status, cudaStream_t s);
+                           int32_t* scratch, int* status, cudaStream_t s);
 cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* tiles, int* status,
                                cudaStream_t s);
 cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, const int32_t* perm,
                           const int32_t* total_rows, uint8_t* xqp, float* xsp, uint32_t* amax,
                           int* status, cudaStream_t s);
+// acts64 / acts16: the routed-row activations with 64-row and 16-row TMA boxes
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
-                               const CUtensorMap& acts, const GemmArgs& a, cudaStream_t s);
+                               const CUtensorMap& acts64, const CUtensorMap& acts16,
+                               const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
-                             const CUtensorMap& acts, const GemmArgs& a, cudaStream_t s);
+                             const CUtensorMap& acts64, const CUtensorMap& acts16,
+                             const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
                            const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s);
 cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t split_stride,

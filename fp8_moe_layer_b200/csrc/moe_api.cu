@@ -61,17 +61,25 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
   p->Rcap = routed + (p->shared ? T : 0);
   p->Rpad = std::max<int64_t>(256, ceil_div(p->Rcap, 256) * 256);
 
-  // token tile: the power of two >= 1.25 x the mean rows of an active expert, in [16, 256]
+  // token tile: the smallest of {16, 32, 64, 128, 192, 256} >= 1.25 x the mean rows of an active
+  // expert. A tile only loads and multiplies its valid rows, so a tile larger than the group
+  // costs shared memory (fewer pipeline stages), not traffic.
   const int64_t active = std::max<int64_t>(1, std::min<int64_t>(E, routed));
   const double mean_rows = double(routed) / double(active);
-  int BN = 16;
-  while (BN < 256 && BN < 1.25 * mean_rows) BN *= 2;
+  static const int kTiles[] = {16, 32, 64, 128, 192, 256};
+  int BN = 256;
+  for (int t : kTiles)
+    if (t >= 1.25 * mean_rows) { BN = t; break; }
+#ifdef MOE_FORCE_BN
+  BN = MOE_FORCE_BN;
+#endif
   p->BN = BN;
 
   // router: 32x32 tiles; split d so that the grid covers about two waves
   const int64_t rtiles = ceil_div(std::max(T, 1), kRouterTile) * ceil_div(E, kRouterTile);
   const int nchunks = (int)ceil_div(d, kRouterTile);
   int rs = (int)std::min<int64_t>(nchunks, std::max<int64_t>(1, ceil_div(2 * kPlanSMs, rtiles)));
+  if (router_uses_mma(E, T)) rs = 1;      // the tensor-core router writes whole logits
   p->r_chunks_per_split = (int)ceil_div(nchunks, rs);
   p->r_splits = (int)ceil_div(nchunks, p->r_chunks_per_split);
 
@@ -95,6 +103,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
   p->off_tiles = take(sizeof(int32_t) * (size_t)(p->G + 2));
   p->off_perm = take(sizeof(int32_t) * (size_t)p->Rpad);
   p->off_inv = take(sizeof(int32_t) * (size_t)routed);
+  p->off_pscr = take(sizeof(int32_t) * 2 * (size_t)permute_blocks(*p) * E);
   p->off_xq = take((size_t)T * d);
   p->off_xs = take(sizeof(float) * (size_t)T);
   p->off_xqp = take((size_t)p->Rpad * d);
@@ -104,6 +113,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
   p->off_aq = take((size_t)p->Rpad * F);
   p->off_s2 = take(sizeof(float) * (size_t)p->Rpad);
   p->off_o = take(sizeof(float) * (size_t)p->g2_splits * p->Rpad * d);
+  p->off_planes = take(router_uses_mma(E, T) ? 3 * sizeof(uint16_t) * (size_t)E * d : 0);
   p->bytes = off;
   return MOE_OK;
 }
@@ -127,10 +137,11 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// e4m3 bytes, 128-byte swizzle, zero fill outside the tensor. dims/strides in elements/bytes,
-// innermost first; strides[i] is the byte stride of dimension i+1.
+// 128-byte swizzle, zero fill outside the tensor. dims/strides in elements/bytes, innermost
+// first; strides[i] is the byte stride of dimension i+1.
 static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                     const uint64_t* strides, const uint32_t* box) {
+                     const uint64_t* strides, const uint32_t* box,
+                     CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -141,9 +152,24 @@ static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
     es[i] = 1;
     if (i + 1 < rank) gs[i] = strides[i];
   }
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), gd, gs, bx, es,
+  return fn(m, dtype, rank, const_cast<void*>(base), gd, gs, bx, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 router weight planes [3][E][d]: box 64 (K) x 128 experts of one plane.
+static bool map_router_planes(CUtensorMap* m, const uint16_t* planes, int E, int d) {
+  const uint64_t dims[3] = {(uint64_t)d, (uint64_t)E, 3};
+  const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)E * d * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return make_map(m, planes, 3, dims, str, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+// bf16 hidden states [T][d]: box 64 (K) x 64 tokens.
+static bool map_hidden(CUtensorMap* m, const uint16_t* hidden, int T, int d) {
+  const uint64_t dims[2] = {(uint64_t)d, (uint64_t)T};
+  const uint64_t str[1] = {(uint64_t)d * 2};
+  const uint32_t box[2] = {64, 64};
+  return make_map(m, hidden, 2, dims, str, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
 // W13 [experts, 2F, d] viewed as [experts][2][F][d]: box 128 (K) x 64 rows of one half.
@@ -187,7 +213,8 @@ static int check_device() {
 struct Ws {
   int* status;
   float *part, *w, *xs, *xsp, *act, *s2, *o;
-  int32_t *ids, *offsets, *tiles, *perm, *inv;
+  uint16_t* planes;
+  int32_t *ids, *offsets, *tiles, *perm, *inv, *pscr;
   uint8_t *xq, *xqp, *aq;
   uint32_t* amax;
 };
@@ -203,6 +230,7 @@ static Ws carve(const Plan& p, void* ws) {
   w.tiles = reinterpret_cast<int32_t*>(b + p.off_tiles);
   w.perm = reinterpret_cast<int32_t*>(b + p.off_perm);
   w.inv = reinterpret_cast<int32_t*>(b + p.off_inv);
+  w.pscr = reinterpret_cast<int32_t*>(b + p.off_pscr);
   w.xq = b + p.off_xq;
   w.xs = reinterpret_cast<float*>(b + p.off_xs);
   w.xqp = b + p.off_xqp;
@@ -212,6 +240,7 @@ static Ws carve(const Plan& p, void* ws) {
   w.aq = b + p.off_aq;
   w.s2 = reinterpret_cast<float*>(b + p.off_s2);
   w.o = reinterpret_cast<float*>(b + p.off_o);
+  w.planes = reinterpret_cast<uint16_t*>(b + p.off_planes);
   return w;
 }
 
@@ -235,6 +264,20 @@ static int check_k(const Plan& p, int k, const int32_t* k_per_token) {
     if ((expr) != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
+// Router logits into w.part for the non-fused paths (tensor cores or CUDA cores).
+static int run_router_logits(const Plan& p, const Ws& w, const uint16_t* hidden,
+                             const float* router_w, cudaStream_t s) {
+  if (router_uses_mma(p)) {
+    CUtensorMap mw, mx;
+    if (!map_router_planes(&mw, w.planes, p.E, p.d) || !map_hidden(&mx, hidden, p.T, p.d))
+      return MOE_ERR_UNSUPPORTED;
+    MOE_CUDA(launch_router_mma(p, router_w, w.planes, mw, mx, w.part, w.status, s));
+    return MOE_OK;
+  }
+  MOE_CUDA(launch_router_logits(p, hidden, router_w, w.part, s));
+  return MOE_OK;
+}
+
 // Grouped FFN core shared by moe_forward and moe_grouped_ffn_fp8: gather, gate/up GEMM +
 // SwiGLU, requantisation, down GEMM into `o` (split partials `split_stride` apart).
 static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* w13_scale,
@@ -242,9 +285,10 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
                    const float* w13s_scale, const uint8_t* w2s, const float* w2s_scale,
                    float* o, size_t split_stride, int64_t o_rows, void* const* ev,
                    cudaStream_t s) {
-  CUtensorMap m13, m13s, mxq, m2, m2s, maq;
+  CUtensorMap m13, m13s, mxq64, mxq16, m2, m2s, maq64, maq16;
   if (!map_w13(&m13, w13, p.E, p.F, p.d) || !map_w2(&m2, w2, p.E, p.d, p.F) ||
-      !map_rows(&mxq, w.xqp, p.Rpad, p.d, p.BN) || !map_rows(&maq, w.aq, p.Rpad, p.F, p.BN))
+      !map_rows(&mxq64, w.xqp, p.Rpad, p.d, 64) || !map_rows(&mxq16, w.xqp, p.Rpad, p.d, 16) ||
+      !map_rows(&maq64, w.aq, p.Rpad, p.F, 64) || !map_rows(&maq16, w.aq, p.Rpad, p.F, 16))
     return MOE_ERR_UNSUPPORTED;
   m13s = m13;
   m2s = m2;
@@ -281,7 +325,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g1.row_amax = w.amax;
   g1.status = w.status;
   record(4);
-  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mxq, g1, s));
+  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mxq64, mxq16, g1, s));
 
   record(5);
   MOE_CUDA(launch_requant(p, w.act, w.amax, total_rows, w.aq, w.s2, s));
@@ -301,7 +345,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g2.out_split_stride = split_stride;
   g2.row_amax = nullptr;
   record(6);
-  MOE_CUDA(launch_gemm_down(p, m2, m2s, maq, g2, s));
+  MOE_CUDA(launch_gemm_down(p, m2, m2s, maq64, maq16, g2, s));
   return MOE_OK;
 }
 
@@ -356,15 +400,21 @@ int moe_route_topk(const moe_dims* dims, const uint16_t* hidden, const float* ro
   MOE_TRY(plan_make(dims->T, dims->d, dims->E, dims->F, dims->k_max, dims->F_shared, &p));
   if (p.T == 0) return MOE_OK;
   if (!hidden || !router_w || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
-  if (!aligned(hidden, 16) || !aligned(router_w, 4)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(router_w, 16)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_k(p, k, k_per_token));
   MOE_TRY(check_ws(p, ws, ws_bytes));
   MOE_TRY(check_device());
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Ws w = carve(p, ws);
-  MOE_CUDA(launch_router_logits(p, hidden, router_w, w.part, s));
+  if (router_is_fused(p)) {
+    MOE_CUDA(launch_route_fused(p, hidden, router_w, router_bias, k, k_per_token, topk_ids, topk_w,
+                                nullptr, nullptr, false, w.status, s));
+    return MOE_OK;
+  }
+  MOE_TRY(run_router_logits(p, w, hidden, router_w, s));
   MOE_CUDA(launch_topk_quant(p, w.part, router_bias, k, k_per_token, topk_ids, topk_w, hidden,
-                             nullptr, nullptr, true, false, w.status, s));
+                             nullptr, nullptr, true, false,
+                             router_uses_mma(p) ? router_w : nullptr, w.status, s));
   return MOE_OK;
 }
 
@@ -384,7 +434,7 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_ids, int32_t k,
   q.shared = false;
   q.G = p.E;
   MOE_CUDA(launch_permute(q, topk_ids, k, k_per_token, expert_offsets, perm_token, inv_row,
-                          w.tiles, w.status, static_cast<cudaStream_t>(stream)));
+                          w.tiles, w.pscr, w.status, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
@@ -411,7 +461,7 @@ int moe_grouped_ffn_fp8(const moe_dims* dims, const uint16_t* hidden, const uint
   q.G = p.E;
   q.Rcap = (int64_t)p.T * p.k_max;
   MOE_CUDA(launch_topk_quant(q, nullptr, nullptr, 1, nullptr, nullptr, nullptr, hidden, w.xq,
-                             w.xs, false, true, w.status, s));
+                             w.xs, false, true, nullptr, w.status, s));
   if (act_scale_out)
     MOE_CUDA(cudaMemcpyAsync(act_scale_out, w.xs, sizeof(float) * p.T, cudaMemcpyDeviceToDevice, s));
   MOE_CUDA(launch_tile_prefix(q, expert_offsets, w.tiles, w.status, s));
@@ -459,8 +509,8 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
   if (p.T == 0) return MOE_OK;
   if (!hidden || !router_w || !w13 || !w13_scale || !w2 || !w2_scale || !y) return MOE_ERR_INVALID_ARG;
   if (p.shared && (!w13_shared || !w13s_scale || !w2_shared || !w2s_scale)) return MOE_ERR_INVALID_ARG;
-  if (!aligned(hidden, 16) || !aligned(w13, 16) || !aligned(w2, 16) || !aligned(y, 16) ||
-      (p.shared && (!aligned(w13_shared, 16) || !aligned(w2_shared, 16))))
+  if (!aligned(hidden, 16) || !aligned(router_w, 16) || !aligned(w13, 16) || !aligned(w2, 16) ||
+      !aligned(y, 16) || (p.shared && (!aligned(w13_shared, 16) || !aligned(w2_shared, 16))))
     return MOE_ERR_INVALID_ARG;
   if (dbg && dbg->y_f32 && !aligned(dbg->y_f32, 16)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_k(p, k, k_per_token));
@@ -475,12 +525,21 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
 
   MOE_CUDA(cudaMemsetAsync(w.status, 0, 16, s));
   record(0);
-  MOE_CUDA(launch_router_logits(p, hidden, router_w, w.part, s));
-  record(1);
-  MOE_CUDA(launch_topk_quant(p, w.part, router_bias, k, k_per_token, w.ids, w.w, hidden, w.xq,
-                             w.xs, true, true, w.status, s));
+  if (router_is_fused(p)) {
+    // one kernel for stages 0 and 1 (stage 1's events bracket nothing)
+    MOE_CUDA(launch_route_fused(p, hidden, router_w, router_bias, k, k_per_token, w.ids, w.w, w.xq,
+                                w.xs, true, w.status, s));
+    record(1);
+  } else {
+    MOE_TRY(run_router_logits(p, w, hidden, router_w, s));
+    record(1);
+    MOE_CUDA(launch_topk_quant(p, w.part, router_bias, k, k_per_token, w.ids, w.w, hidden, w.xq,
+                               w.xs, true, true, router_uses_mma(p) ? router_w : nullptr,
+                               w.status, s));
+  }
   record(2);
-  MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.status, s));
+  MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
+                          w.status, s));
   const size_t split_stride = (size_t)p.Rpad * p.d;
   MOE_TRY(run_ffn(p, w, w13, w13_scale, w2, w2_scale, w13_shared, w13s_scale, w2_shared,
                   w2s_scale, w.o, split_stride, p.Rcap, ev, s));

@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
     int E, int has_shared, int BN, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
     int32_t* __restrict__ inv, int32_t* __restrict__ tiles, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   extern __shared__ int hist[];                  // [kPermWarps][E]
   __shared__ int warp_sums[33];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -141,10 +143,161 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     for (int t = threadIdx.x; t < T; t += kPermThreads) perm[total_rows + t] = t;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Multi-block grouping for large T * k_max. Block b owns tokens [b*chunk, (b+1)*chunk) and its
+// warps own contiguous sub-ranges, so (block, warp, batch, lane) order is token order:
+//   count:   per-block expert counts -> bcount[b][e]
+//   scan:    offsets, per-block bases bbase[b][e] = offsets[e] + sum_{b'<b} bcount[b'][e],
+//            GEMM tile prefix (one block)
+//   scatter: per-warp cursors = bbase[b][e] + counts of the block's earlier warps, then the same
+//            stable __match_any_sync ranking as the single-block kernel.
+constexpr int kPermBlkThreads = 256;
+constexpr int kPermBlkWarps = kPermBlkThreads / 32;
+
+__device__ __forceinline__ void warp_range(int T, int k_max, int blocks, long long& i_begin,
+                                           long long& i_end) {
+  const int bchunk = (T + blocks - 1) / blocks;
+  const int bt0 = min(T, (int)blockIdx.x * bchunk), bt1 = min(T, bt0 + bchunk);
+  const int wchunk = (bt1 - bt0 + kPermBlkWarps - 1) / kPermBlkWarps;
+  const int warp = threadIdx.x >> 5;
+  const int t0 = min(bt1, bt0 + warp * wchunk), t1 = min(bt1, t0 + wchunk);
+  i_begin = (long long)t0 * k_max;
+  i_end = (long long)t1 * k_max;
+}
+
+// shared-memory per-warp counts of this block's (token, slot) pairs
+__device__ __forceinline__ void block_warp_counts(const int32_t* ids, int T, int k_max, int k,
+                                                  const int32_t* k_per_token, int E, int blocks,
+                                                  int* whist, int* status, bool flag) {
+  for (int i = threadIdx.x; i < kPermBlkWarps * E; i += kPermBlkThreads) whist[i] = 0;
+  __syncthreads();
+  long long i_begin, i_end;
+  warp_range(T, k_max, blocks, i_begin, i_end);
+  int* my = whist + (threadIdx.x >> 5) * E;
+  const int lane = threadIdx.x & 31;
+  for (long long base = i_begin; base < i_end; base += 32) {
+    const long long idx = base + lane;
+    if (idx < i_end) {
+      const int t = (int)(idx / k_max), j = (int)(idx % k_max);
+      const int kt = k_per_token ? k_per_token[t] : k;
+      if (j < kt) {
+        const int e = ids[idx];
+        if (e >= 0 && e < E) atomicAdd(&my[e], 1);
+        else if (flag) report(status, kStatusDeviceCheck, kWherePermute, t);
+      }
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kPermBlkThreads) permute_count_kernel(
+    const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
+    int E, int32_t* __restrict__ bcount, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  extern __shared__ int whist[];
+  block_warp_counts(ids, T, k_max, k, k_per_token, E, gridDim.x, whist, status, true);
+  for (int e = threadIdx.x; e < E; e += kPermBlkThreads) {
+    int c = 0;
+    for (int w = 0; w < kPermBlkWarps; ++w) c += whist[w * E + e];
+    bcount[(size_t)blockIdx.x * E + e] = c;
+  }
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(
+    const int32_t* __restrict__ bcount, int blocks, int T, int E, int has_shared, int BN,
+    int32_t* __restrict__ bbase, int32_t* __restrict__ offsets, int32_t* __restrict__ tiles) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  __shared__ int warp_sums[33];
+  const int e = threadIdx.x;                 // E <= 1024 = blockDim
+  int cnt = 0;
+  if (e < E)
+    for (int b = 0; b < blocks; ++b) cnt += bcount[(size_t)b * E + e];
+  int total_rows = 0, total_tiles = 0;
+  const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
+  if (e < E) {
+    offsets[e] = off;
+    int run = off;
+    for (int b = 0; b < blocks; ++b) {
+      bbase[(size_t)b * E + e] = run;
+      run += bcount[(size_t)b * E + e];
+    }
+  }
+  const int nt = e < E ? (cnt + BN - 1) / BN : 0;
+  const int toff = block_exclusive_scan(nt, warp_sums, total_tiles);
+  if (e < E) tiles[e] = toff;
+  if (threadIdx.x == 0) {
+    offsets[E] = total_rows;
+    tiles[E] = total_tiles;
+    if (has_shared) {
+      offsets[E + 1] = total_rows + T;
+      tiles[E + 1] = total_tiles + (T + BN - 1) / BN;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPermBlkThreads) permute_scatter_kernel(
+    const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
+    int E, int has_shared, const int32_t* __restrict__ bbase, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  extern __shared__ int whist[];
+  block_warp_counts(ids, T, k_max, k, k_per_token, E, gridDim.x, whist, nullptr, false);
+  // per-warp cursors: the block's base plus the counts of its earlier warps
+  for (int e = threadIdx.x; e < E; e += kPermBlkThreads) {
+    int run = bbase[(size_t)blockIdx.x * E + e];
+    for (int w = 0; w < kPermBlkWarps; ++w) {
+      const int c = whist[w * E + e];
+      whist[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  long long i_begin, i_end;
+  warp_range(T, k_max, gridDim.x, i_begin, i_end);
+  int* my = whist + (threadIdx.x >> 5) * E;
+  const int lane = threadIdx.x & 31;
+  for (long long base = i_begin; base < i_end; base += 32) {
+    const long long idx = base + lane;
+    bool valid = false;
+    int t = 0, e = -1;
+    if (idx < i_end) {
+      t = (int)(idx / k_max);
+      const int j = (int)(idx % k_max);
+      const int kt = k_per_token ? k_per_token[t] : k;
+      if (j < kt) {
+        e = ids[idx];
+        valid = e >= 0 && e < E;
+      }
+      if (!valid) inv[idx] = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : E + lane);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int cursor = valid ? my[e] : 0;
+    __syncwarp();
+    if (valid) {
+      const int r = cursor + rank;
+      perm[r] = t;
+      inv[idx] = r;
+      if (rank == 0) my[e] = cursor + __popc(peers);
+    }
+    __syncwarp();
+  }
+  if (has_shared) {
+    const int R = offsets[E];
+    for (int t = blockIdx.x * kPermBlkThreads + threadIdx.x; t < T; t += gridDim.x * kPermBlkThreads)
+      perm[R + t] = t;
+  }
+}
+
 // For caller-provided offsets (split entry point): validate and build the GEMM tile prefix.
 __global__ void __launch_bounds__(kPermThreads) tile_prefix_kernel(
     const int32_t* __restrict__ offsets, int E, int64_t rcap, int BN, int32_t* __restrict__ tiles,
     int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   __shared__ int warp_sums[33];
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
@@ -176,6 +329,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
     const uint8_t* __restrict__ xq, const float* __restrict__ xs, const int32_t* __restrict__ perm,
     const int32_t* __restrict__ total_rows, int64_t rcap, int T, int d, uint8_t* __restrict__ xqp,
     float* __restrict__ xsp, uint32_t* __restrict__ amax, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
   const int lane = threadIdx.x & 31;
   const int nv = d / 16;
@@ -197,26 +352,50 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
   }
 }
 
+// Blocks of the multi-block grouping: about 1024 (token, slot) pairs each, at most 4 per SM.
+int permute_blocks(const Plan& p) {
+  const long long slots = (long long)p.T * p.k_max;
+  if (slots <= 8192) return 1;
+  return (int)std::min<long long>((slots + 1023) / 1024, 4LL * 148);
+}
+
 cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
-                           int* status, cudaStream_t s) {
-  const size_t smem = sizeof(int) * kPermWarps * p.E;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kPermWarps * kMaxExperts * (int)sizeof(int));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+                           int32_t* scratch, int* status, cudaStream_t s) {
+  const int blocks = permute_blocks(p);
+  if (blocks == 1) {
+    const size_t smem = sizeof(int) * kPermWarps * p.E;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    if (dev < 64 && !attr_set[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(permute_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kPermWarps * kMaxExperts * (int)sizeof(int));
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), smem, s, ids, p.T, p.k_max, k, k_per_token, p.E,
+                                                 p.shared ? 1 : 0, p.BN, offsets, perm, inv, tiles,
+                                                 status);
+    return cudaGetLastError();
   }
-  permute_kernel<<<1, kPermThreads, smem, s>>>(ids, p.T, p.k_max, k, k_per_token, p.E,
-                                               p.shared ? 1 : 0, p.BN, offsets, perm, inv, tiles,
-                                               status);
+  int32_t* bcount = scratch;
+  int32_t* bbase = scratch + (size_t)blocks * p.E;
+  const size_t smem = sizeof(int) * kPermBlkWarps * p.E;   // <= 32 KB
+  launch_pdl(permute_count_kernel, dim3(blocks), dim3(kPermBlkThreads), smem, s, ids, p.T, p.k_max, k, k_per_token,
+                                                             p.E, bcount, status);
+  launch_pdl(permute_scan_kernel, dim3(1), dim3(kPermThreads), 0, s, bcount, blocks, p.T, p.E, p.shared ? 1 : 0, p.BN,
+                                                 bbase, offsets, tiles);
+  launch_pdl(permute_scatter_kernel, dim3(blocks), dim3(kPermBlkThreads), smem, s, ids, p.T, p.k_max, k, k_per_token,
+                                                               p.E, p.shared ? 1 : 0, bbase,
+                                                               offsets, perm, inv);
   return cudaGetLastError();
 }
 
 cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* tiles, int* status,
                                cudaStream_t s) {
-  tile_prefix_kernel<<<1, kPermThreads, 0, s>>>(offsets, p.E, (int64_t)p.T * p.k_max, p.BN, tiles,
+  launch_pdl(tile_prefix_kernel, dim3(1), dim3(kPermThreads), 0, s, offsets, p.E, (int64_t)p.T * p.k_max, p.BN, tiles,
                                                 status);
   return cudaGetLastError();
 }
@@ -226,7 +405,7 @@ cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, con
                           int* status, cudaStream_t s) {
   const int64_t blocks_needed = (p.Rcap + 7) / 8;
   const int grid = (int)std::min<int64_t>(std::max<int64_t>(blocks_needed, 1), 8LL * num_sms());
-  gather_rows_kernel<<<grid, 256, 0, s>>>(xq, xs, perm, total_rows, p.Rcap, p.T, p.d, xqp, xsp,
+  launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, s, xq, xs, perm, total_rows, p.Rcap, p.T, p.d, xqp, xsp,
                                           amax, status);
   return cudaGetLastError();
 }

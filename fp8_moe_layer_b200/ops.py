@@ -46,12 +46,12 @@ class MoEError(RuntimeError):
         super().__init__(f"{where}: {status_string(status)} (status {status})")
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m fp8_moe_layer_b200.build` "
+            f"{path} is missing: build it with `python -m fp8_moe_layer_b200.build` "
             "(nvcc, sm_100a). The FP8 MoE layer has no other implementation.")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     dims_p = ctypes.POINTER(MoEDims)
     sig = {

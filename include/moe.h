@@ -21,6 +21,8 @@
  *     argument says otherwise; layouts are dense row-major with the last index contiguous.
  *   - bf16 tensors are passed as uint16_t bit patterns; e4m3 tensors as uint8_t codes (OCP FP8
  *     e4m3fn: bias 7, 3 mantissa bits, max 448, 0x7F/0xFF NaN).
+ *   - hidden, router_w, w13, w2 (and the shared expert's weights), y and every fp32 output read
+ *     or written with 128-bit accesses must be 16-byte aligned (torch allocations are).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every call is
  *     asynchronous on that stream and never synchronises it, except moe_device_status.
  *   - Ownership: the caller allocates and frees every buffer, including the workspace `ws`

@@ -9,8 +9,11 @@ from fp8_moe_layer_b200 import inputs as I
 from oracle import moe_oracle as O
 
 # ----------------------------------------------------------------------------- tolerances
-# Routing weights: fp32 softmax of fp32 logits against the float64 oracle.
-WEIGHT_ATOL = 2e-6
+# Routing weights: fp32 softmax of fp32 logits against the float64 oracle. |dw_j| <= 2 w_j
+# max|dl|, and the rounding error of an fp32 dot product grows like sqrt(d): 2e-6 at d <= 512,
+# scaled by sqrt(d / 512) above (7.5e-6 at d = 7168).
+def weight_atol(d: int) -> float:
+    return 2e-6 * max(1.0, (d / 512.0) ** 0.5)
 # Output of the layer (bf16). The bar is max |err| <= 2e-2 and relative L2 <= 1e-2:
 #  (i)   the fp32 sum before its bf16 rounding is within 2e-2 of the float64 result;
 #  (ii)  the bf16 output is within 2e-2 + half a bf16 ulp of it (one more rounding of (i));
@@ -74,15 +77,17 @@ def order_tie_tokens(logits: np.ndarray, k_t: np.ndarray, gap: float = NEAR_TIE)
     return np.asarray(out, dtype=np.int64)
 
 
-def check_routing(gpu_ids: np.ndarray, gpu_w: np.ndarray, ref: dict):
+def check_routing(gpu_ids: np.ndarray, gpu_w: np.ndarray, ref: dict, d: int):
     """Routing parity.
-    * Tokens without any near tie: ids bit-exact (set and slot order), weights within WEIGHT_ATOL.
+    * Tokens without any near tie: ids bit-exact (set and slot order), weights within
+      weight_atol(d).
     * Near tie at the k-th place (k-th and (k+1)-th oracle logits within NEAR_TIE): the GPU's
       choice must be a valid top-k -- k_t distinct experts, each within NEAR_TIE of the k-th.
     * Near tie inside the selection only: the SET is bit-exact, the GPU order is descending in
       the oracle logits up to NEAR_TIE, and each expert's weight matches.
     Returns (boundary near ties, how many of them chose differently, order-only near ties)."""
     logits, ids, w, k_t = ref["logits"], ref["topk_ids"], ref["topk_w"], ref["k_t"]
+    atol = weight_atol(d)
     near = set(O.near_tie_tokens(logits, k_t, NEAR_TIE).tolist())
     order = set(order_tie_tokens(logits, k_t, NEAR_TIE).tolist()) - near
     differed = 0
@@ -101,10 +106,10 @@ def check_routing(gpu_ids: np.ndarray, gpu_w: np.ndarray, ref: dict):
             assert set(sel.tolist()) == set(ids[t, :kt].tolist()), t
             assert np.all(np.diff(logits[t, sel]) <= NEAR_TIE), t
             ref_w = dict(zip(ids[t, :kt].tolist(), w[t, :kt].tolist()))
-            assert max(abs(gpu_w[t, j] - ref_w[int(e)]) for j, e in enumerate(sel)) <= WEIGHT_ATOL
+            assert max(abs(gpu_w[t, j] - ref_w[int(e)]) for j, e in enumerate(sel)) <= atol
             continue
         assert np.array_equal(sel, ids[t, :kt]), (t, gpu_ids[t], ids[t])
-        assert np.abs(gpu_w[t, :kt] - w[t, :kt]).max() <= WEIGHT_ATOL, (t, gpu_w[t], w[t])
+        assert np.abs(gpu_w[t, :kt] - w[t, :kt]).max() <= atol, (t, gpu_w[t], w[t])
     return len(near), differed, len(order)
 
 

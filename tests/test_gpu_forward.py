@@ -35,7 +35,7 @@ def forward_and_check(ops, inp, sample=None, seed=0):
     k_t = O.token_k(s.T, s.k, H.np_(inp.k_per_token))
     ids = O.select_topk(logits, k_t, s.k_max)
     route_ref = dict(logits=logits, topk_ids=ids, topk_w=O.routing_weights(logits, ids), k_t=k_t)
-    n_near, differed, n_order = H.check_routing(gpu["topk_ids"], gpu["topk_w"], route_ref)
+    n_near, differed, n_order = H.check_routing(gpu["topk_ids"], gpu["topk_w"], route_ref, s.d)
     H.check_grouping(gpu["expert_offsets"], gpu["perm_token"], gpu["inv_row"],
                      gpu["topk_ids"], k_t, s.E)
 

@@ -12,6 +12,9 @@ pytestmark = pytest.mark.gpu
 
 ROUTE_SHAPES = [
     I.WORKLOADS["tiny_T16"],
+    I.MoEShape("cuda_core_router", 37, 256, 64, 64, 6, 6, zipf_s=0.8),     # E > 32, T < 64
+    I.MoEShape("mma_router_ragged_E", 100, 320, 48, 64, 4, 4),              # E % 128 != 0
+    I.MoEShape("mma_router_E33", 65, 128, 33, 64, 3, 3),
     I.MoEShape("ragged", 37, 256, 6, 64, 2, 2),
     I.MoEShape("k_equals_E", 19, 128, 5, 64, 5, 5),
     I.WORKLOADS["qwen3_T64"],
@@ -50,7 +53,7 @@ def test_route_topk_matches_oracle(ops, shape):
     ref = _oracle_route(shape, hidden, rw, rb, kpt)
     c = lambda t: None if t is None else t.cuda()
     ids, w = ops.moe_route_topk(c(hidden), c(rw), c(rb), shape.k, c(kpt), shape.k_max)
-    n_near, differed, n_order = H.check_routing(H.np_(ids), H.np_(w), ref)
+    n_near, differed, n_order = H.check_routing(H.np_(ids), H.np_(w), ref, shape.d)
     print(f"{shape.name}: near-tie tokens {n_near}, differing among them {differed}, "
           f"order-only ties {n_order}")
 
