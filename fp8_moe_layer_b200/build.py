@@ -13,7 +13,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8moe.so")
-SOURCES = ["moe_api.cu", "route.cu", "router_mma.cu", "permute.cu", "gemm.cu", "combine.cu"]
+SOURCES = ["moe_api.cu", "route.cu", "router_mma.cu", "permute.cu", "gemm.cu", "combine.cu",
+           "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -66,6 +66,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_combine": (ctypes.c_int, [dims_p, vp, vp, vp, vp, vp, vp, vp]),
         "moe_forward": (ctypes.c_int, [dims_p, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                        vp, vp, vp, sz, vp, ctypes.POINTER(MoEDebugOut)]),
+        "moe_route_topk_noalloc": (ctypes.c_int, [dims_p, vp, vp, vp, i32, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

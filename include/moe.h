@@ -161,6 +161,27 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                 const uint8_t* w2_shared, const float* w2s_scale, uint16_t* y, void* ws,
                 size_t ws_bytes, void* stream, const moe_debug_out* dbg);
 
+/* Router top-k without a workspace, for callers that cannot allocate device memory: an engine
+ * that has already handed all device memory to its own pools, or a step that runs where
+ * allocating is not allowed. The pages describing the method have no counterpart to this entry
+ * point; it returns the same routing decision as moe_route_topk (same arguments, minus the
+ * workspace), computed with the CUDA-core router.
+ *   Scratch: one fixed device array of MOE_NOALLOC_SCRATCH_BYTES owned by this library, which
+ *   every GPU that loads the library keeps until the process exits. It holds the partial router
+ *   logits, 4 * T * E * splits bytes (splits = the number of pieces d is cut into so that the
+ *   logits kernel fills the GPU; none at all for E <= 32); a larger shape returns
+ *   MOE_ERR_UNSUPPORTED and launches nothing.
+ *   The first call on a device looks up the array's device address (with that device current);
+ *   make that first call before any stream capture.
+ *   Every call uses the same array, and each call overwrites the partial logits it reads, so
+ *   nothing in it needs clearing. Calls that overlap on one GPU (on different streams, or from
+ *   several host threads) race for it and can return wrong results: serialise them.
+ *   A k_t outside [1, min(E, k_max)] is clamped without a report (there is no status word). */
+#define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int moe_route_topk_noalloc(const moe_dims* dims, const uint16_t* hidden, const float* router_w,
+                           const float* router_bias, int32_t k, const int32_t* k_per_token,
+                           int32_t* topk_ids, float* topk_w, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
