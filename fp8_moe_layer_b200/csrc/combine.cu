@@ -14,6 +14,8 @@
 namespace moe {
 
 // s2[r] = amax[r] / 448 (IEEE fp32; 1 if 0); aq[r, f] = e4m3_rne_satfinite(act[r, f] / s2[r]).
+// The row max is already complete (from the gate/up epilogue), so every 4-element chunk of every
+// row is independent: a flat grid-stride loop over (row, chunk), 128-bit loads, 32-bit stores.
 __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ act,
                                                       const uint32_t* __restrict__ amax,
                                                       const int32_t* __restrict__ total_rows,
@@ -22,19 +24,70 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
                                                       float* __restrict__ s2) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
+  const int64_t R = min((int64_t)max(*total_rows, 0), rcap);
   const int nv = F / 4;
-  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+  const int64_t n = R * nv;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / nv;
+    const int c = (int)(i - r * nv);
     const float am = __uint_as_float(amax[r]);
     const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+    if (c == 0) s2[r] = sc;
+    const float4 v = reinterpret_cast<const float4*>(act + r * F)[c];
+    reinterpret_cast<uint32_t*>(aq + r * F)[c] =
+        static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.x, sc), __fdiv_rn(v.y, sc))) |
+        (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.z, sc), __fdiv_rn(v.w, sc))) << 16);
+  }
+}
+
+// K-split gate/up: per routed row, gate[f] = sum_s h[s][r][f], up[f] = sum_s h[s][r][F + f]
+// (split order fixed), act = silu(gate) * up, s2 = amax|act| / 448 (IEEE fp32; 1 if 0),
+// aq = e4m3(act / s2). One block per row; act is recomputed in the second pass instead of stored.
+__global__ void __launch_bounds__(256) swiglu_requant_kernel(
+    const float* __restrict__ h, int splits, size_t split_stride,
+    const int32_t* __restrict__ total_rows, int64_t rcap, int F, uint8_t* __restrict__ aq,
+    float* __restrict__ s2) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  __shared__ float red[8];
+  const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
+  const int nv = F / 4;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+    auto act4 = [&](int i) {
+      const float4* g4 = reinterpret_cast<const float4*>(h + (size_t)r * 2 * F);
+      const float4* u4 = reinterpret_cast<const float4*>(h + (size_t)r * 2 * F + F);
+      float4 g = g4[i], u = u4[i];
+      for (int sp = 1; sp < splits; ++sp) {
+        const float4 gs = reinterpret_cast<const float4*>(h + sp * split_stride + (size_t)r * 2 * F)[i];
+        const float4 us = reinterpret_cast<const float4*>(h + sp * split_stride + (size_t)r * 2 * F + F)[i];
+        g.x += gs.x; g.y += gs.y; g.z += gs.z; g.w += gs.w;
+        u.x += us.x; u.y += us.y; u.z += us.z; u.w += us.w;
+      }
+      return make_float4(silu(g.x) * u.x, silu(g.y) * u.y, silu(g.z) * u.z, silu(g.w) * u.w);
+    };
+    float amax = 0.f;
+    for (int i = threadIdx.x; i < nv; i += blockDim.x) {
+      const float4 a = act4(i);
+      amax = fmaxf(fmaxf(amax, fmaxf(fabsf(a.x), fabsf(a.y))), fmaxf(fabsf(a.z), fabsf(a.w)));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    float am = red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) am = fmaxf(am, red[w]);
+    const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
     if (threadIdx.x == 0) s2[r] = sc;
-    const float4* src = reinterpret_cast<const float4*>(act + (size_t)r * F);
     uint32_t* dst = reinterpret_cast<uint32_t*>(aq + (size_t)r * F);
     for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-      const float4 v = src[i];
+      const float4 v = act4(i);
       dst[i] = static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.x, sc), __fdiv_rn(v.y, sc))) |
                (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.z, sc), __fdiv_rn(v.w, sc))) << 16);
     }
+    __syncthreads();                                   // red[] is reused by the next row
   }
 }
 
@@ -125,7 +178,19 @@ static int row_grid(int64_t rows) {
 
 cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
                            const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s) {
-  launch_pdl(requant_kernel, dim3(row_grid(p.Rcap)), dim3(256), 0, s, act, amax, total_rows, p.Rcap, p.F, aq, s2);
+  const int64_t chunks = p.Rcap * (p.F / 4);
+  const int grid = (int)std::min<int64_t>(std::max<int64_t>((chunks + 255) / 256, 1),
+                                          16LL * num_sms());
+  launch_pdl(requant_kernel, dim3(grid), dim3(256), 0, s, act, amax, total_rows, p.Rcap, p.F, aq,
+             s2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_requant(const Plan& p, const float* h, int splits, size_t split_stride,
+                                  const int32_t* total_rows, uint8_t* aq, float* s2,
+                                  cudaStream_t s) {
+  launch_pdl(swiglu_requant_kernel, dim3(row_grid(p.Rcap)), dim3(256), 0, s, h, splits,
+             split_stride, total_rows, p.Rcap, p.F, aq, s2);
   return cudaGetLastError();
 }
 

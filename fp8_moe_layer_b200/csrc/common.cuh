@@ -242,6 +242,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// silu(g) = g / (1 + e^-g) with the fast exponential and division; the exponent is clamped so the
+// denominator stays finite (silu(g) < 1e-30 in magnitude below g = -80).
+__device__ __forceinline__ float silu(float g) {
+  return __fdividef(g, 1.f + __expf(fminf(-g, 80.f)));
+}
+
 // ---------------------------------------------------------------- conversions
 // Two fp32 values to two e4m3 codes (round to nearest even, saturate to +-448); `lo` lands in the
 // lower byte.

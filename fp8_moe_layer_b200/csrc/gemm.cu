@@ -32,19 +32,22 @@
 
 namespace moe {
 
-template <int BN, bool GATEUP>
+template <int BN, int MODE>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int A_BYTES = BM * kBK;
   static constexpr int B_BYTES = BN * kBK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int XCHG_LD = 33;                       // padded row of the exchange buffer
-  static constexpr int XCHG_BYTES = GATEUP ? 128 * XCHG_LD * 4 : 0;
+  static constexpr int XCHG_BYTES = MODE == kModeSwiGLU ? 128 * XCHG_LD * 4 : 0;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_MAX = 232448;                  // 227 KB per block
-  static constexpr int STAGES_FIT = (SMEM_MAX - 1024 - XCHG_BYTES - BAR_BYTES) / STAGE_BYTES;
+  // group offsets and tile prefix of up to kMaxExperts + 1 groups, cached in shared memory
+  static constexpr int TABLE_BYTES = 2 * (kMaxExperts + 2) * 4;
+  static constexpr int STAGES_FIT =
+      (SMEM_MAX - 1024 - XCHG_BYTES - BAR_BYTES - TABLE_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCHG_BYTES + BAR_BYTES;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCHG_BYTES + BAR_BYTES + TABLE_BYTES;
   // two accumulator buffers; the allocation is a power of two >= 32 columns
   static constexpr int TMEM_COLS = 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128
                                    : 2 * BN <= 256 ? 256 : 512;
@@ -54,41 +57,43 @@ struct GemmCfg {
   static_assert(BN % CW == 0, "epilogue chunks");
 };
 
-// tile -> (group g, m-tile, K-split s, n-tile). Group g covers tiles
-// [MS * prefix[g], MS * prefix[g+1]) with MS = m_tiles * splits; inside it n runs fastest.
-__device__ __forceinline__ void decode_tile(const GemmArgs& a, int tile, int& g, int& m, int& n,
+// The tile list, read from shared-memory copies of the group offsets and the tile prefix (a tile
+// boundary then costs a few shared-memory loads instead of a chain of global ones).
+struct TileTable {
+  const int* off;   // [G+1] first routed row of each group
+  const int* tp;    // [G+1] prefix over groups of the token tiles
+  int G, ms, splits;
+};
+
+// tile -> (group g, m-tile, K-split s, n-tile). Group g covers tiles [ms * tp[g], ms * tp[g+1])
+// with ms = m_tiles * splits; inside it n runs fastest.
+__device__ __forceinline__ void decode_tile(const TileTable& tt, int tile, int& g, int& m, int& n,
                                             int& s) {
-  const int ms = a.m_tiles * a.splits;
-  const int v = tile / ms;
-  int lo = 0, hi = a.G - 1;
+  const int v = tile / tt.ms;
+  int lo = 0, hi = tt.G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (a.tile_prefix[mid] <= v) lo = mid;
+    if (tt.tp[mid] <= v) lo = mid;
     else hi = mid - 1;
   }
   g = lo;
-  const int local = tile - ms * a.tile_prefix[g];
-  const int nt = a.tile_prefix[g + 1] - a.tile_prefix[g];
+  const int local = tile - tt.ms * tt.tp[g];
+  const int nt = tt.tp[g + 1] - tt.tp[g];
   n = local % nt;
   const int rest = local / nt;
-  s = rest % a.splits;
-  m = rest / a.splits;
+  s = rest % tt.splits;
+  m = rest / tt.splits;
 }
 
 // Valid token rows of the tile starting at row0 of group g, rounded up to a multiple of 16.
 template <int BN>
-__device__ __forceinline__ int tile_rows16(const GemmArgs& a, int g, int row0) {
-  const int rows = min(BN, a.group_offsets[g + 1] - row0);
+__device__ __forceinline__ int tile_rows16(const TileTable& tt, int g, int row0) {
+  const int rows = min(BN, tt.off[g + 1] - row0);
   return (rows + 15) & ~15;
 }
 
-// silu(g) = g / (1 + e^-g) with the fast exponential and division; the exponent is clamped so the
-// denominator stays finite (silu(g) < 1e-30 in magnitude below g = -80).
-__device__ __forceinline__ float silu(float g) {
-  return __fdividef(g, 1.f + __expf(fminf(-g, 80.f)));
-}
 
-template <int BN, bool GATEUP>
+template <int BN, int MODE>
 __global__ void __launch_bounds__(256, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_a_shared,
@@ -96,8 +101,9 @@ __global__ void __launch_bounds__(256, 1)
                         const __grid_constant__ CUtensorMap map_b16, const GemmArgs args) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  using C = GemmCfg<BN, GATEUP>;
-  constexpr int kWhere = GATEUP ? kWhereGemm1 : kWhereGemm2;
+  using C = GemmCfg<BN, MODE>;
+  constexpr bool kGateUp = MODE != kModeDown;     // A tile = 64 gate rows + the 64 up rows
+  constexpr int kWhere = kGateUp ? kWhereGemm1 : kWhereGemm2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;
@@ -112,6 +118,13 @@ __global__ void __launch_bounds__(256, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total_tiles = args.m_tiles * args.splits * args.tile_prefix[args.G];
   if (static_cast<int>(blockIdx.x) >= total_tiles) return;
+  int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
+  int* s_tp = s_off + (kMaxExperts + 2);
+  for (int i = threadIdx.x; i <= args.G; i += blockDim.x) {
+    s_off[i] = args.group_offsets[i];
+    s_tp[i] = args.tile_prefix[i];
+  }
+  const TileTable tt{s_off, s_tp, args.G, args.m_tiles * args.splits, args.splits};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -148,9 +161,9 @@ __global__ void __launch_bounds__(256, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         int g, m, n, s;
-        decode_tile(args, tile, g, m, n, s);
-        const int row0 = args.group_offsets[g] + n * BN;
-        const int rows16 = tile_rows16<BN>(args, g, row0);   // valid token rows, rounded to 16
+        decode_tile(tt, tile, g, m, n, s);
+        const int row0 = tt.off[g] + n * BN;
+        const int rows16 = tile_rows16<BN>(tt, g, row0);   // valid token rows, rounded to 16
         const uint32_t stage_bytes = C::A_BYTES + rows16 * kBK;
         const int kb0 = s * args.kb_per_split;
         const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
@@ -165,7 +178,7 @@ __global__ void __launch_bounds__(256, 1)
           }
           uint8_t* sa = stages + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], stage_bytes);
-          if (GATEUP) {
+          if (kGateUp) {
             tma_load_4d(sa, ma, &full[stage], kb * kBK, m * 64, 0, ga, pol_w);
             tma_load_4d(sa + C::A_BYTES / 2, ma, &full[stage], kb * kBK, m * 64, 1, ga, pol_w);
           } else {
@@ -206,12 +219,12 @@ __global__ void __launch_bounds__(256, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
         int g, m, n, s;
-        decode_tile(args, tile, g, m, n, s);
+        decode_tile(tt, tile, g, m, n, s);
         const int kb0 = s * args.kb_per_split;
         const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
         // MMA N = the tile's valid rows rounded up to 16 (M = 128 takes N = 16 .. 256 by 16)
         const uint32_t idesc =
-            idesc_e4m3_f32(128, tile_rows16<BN>(args, g, args.group_offsets[g] + n * BN));
+            idesc_e4m3_f32(128, tile_rows16<BN>(tt, g, tt.off[g] + n * BN));
         const int ab = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         if (!mbar_wait(&tempty[ab], aph ^ 1u)) {
@@ -255,7 +268,7 @@ __global__ void __launch_bounds__(256, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
       int g, m, n, s;
-      decode_tile(args, tile, g, m, n, s);
+      decode_tile(tt, tile, g, m, n, s);
       const int ab = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       if (!bad) {
@@ -264,12 +277,12 @@ __global__ void __launch_bounds__(256, 1)
         if (bad && lane == 0) report(args.status, kStatusDeviceTimeout, kWhere, 5);
       }
       tc_fence_after_sync();
-      const int row0 = args.group_offsets[g] + n * BN;
-      const int nvalid = min(BN, args.group_offsets[g + 1] - row0);
+      const int row0 = tt.off[g] + n * BN;
+      const int nvalid = min(BN, tt.off[g + 1] - row0);
       const bool sh = g >= args.E_routed;
       const float* wsc = sh ? args.w_scale_shared : args.w_scale + (size_t)g * args.w_scale_ld;
       const uint32_t tbase = tmem_base + ab * BN + (static_cast<uint32_t>(32 * q) << 16);
-      if constexpr (GATEUP) {
+      if constexpr (MODE == kModeSwiGLU) {
         // TMEM lane 32q+i holds gate row (q<2) or up row (q>=2) 32*(q&1)+i of this 64-row half
         // pair. Step 1: every warp parks its rows (scaled by the weight scale) in smem.
         // Step 2: thread (q, lane) takes token column `lane` and the 16 features 16q .. 16q+15:
@@ -311,6 +324,26 @@ __global__ void __launch_bounds__(256, 1)
           }
           named_bar_sync(1, 128);
         }
+      } else if constexpr (MODE == kModeGateUpPartial) {
+        // K-split gate/up: scaled partial sums of gate (columns [0, F)) and up ([F, 2F)) rows
+        const int half = q >> 1;
+        const int frow = m * 64 + 32 * (q & 1) + lane;
+        const bool valid_row = frow < args.M_valid;
+        const float wsv = valid_row ? wsc[half * args.M_valid + frow] : 0.f;
+        const int col = half * args.M_valid + frow;
+        float* outp = args.out + (size_t)s * args.out_split_stride;
+        for (int c0 = 0; !bad && c0 < nvalid; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tbase + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int nn = c0 + c;
+            if (nn < nvalid && valid_row)
+              outp[(size_t)(row0 + nn) * args.out_ld + col] =
+                  __uint_as_float(r[c]) * args.row_scale[row0 + nn] * wsv;
+          }
+        }
       } else {
         const int i = m * 128 + 32 * q + lane;         // output channel
         const float wsv = i < args.M_valid ? wsc[i] : 0.f;
@@ -343,50 +376,55 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 namespace {
-template <int BN, bool GATEUP>
+template <int BN, int MODE>
 cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& ash, const CUtensorMap& b64,
                           const CUtensorMap& b16, const GemmArgs& args, cudaStream_t s) {
-  using C = GemmCfg<BN, GATEUP>;
+  using C = GemmCfg<BN, MODE>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 64 && !attr_done[dev]) {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel<BN, GATEUP>,
+    err = cudaFuncSetAttribute(grouped_gemm_kernel<BN, MODE>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
     attr_done[dev] = true;
   }
-  launch_pdl(grouped_gemm_kernel<BN, GATEUP>, dim3(num_sms()), dim3(256), C::SMEM, s, a, ash, b64, b16, args);
+  launch_pdl(grouped_gemm_kernel<BN, MODE>, dim3(num_sms()), dim3(256), C::SMEM, s, a, ash, b64, b16, args);
   return cudaGetLastError();
 }
 
-template <bool GATEUP>
+template <int MODE>
 cudaError_t launch_by_bn(int BN, const CUtensorMap& a, const CUtensorMap& ash,
                          const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& args,
                          cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_gemm_t<16, GATEUP>(a, ash, b64, b16, args, s);
-    case 32: return launch_gemm_t<32, GATEUP>(a, ash, b64, b16, args, s);
-    case 64: return launch_gemm_t<64, GATEUP>(a, ash, b64, b16, args, s);
-    case 128: return launch_gemm_t<128, GATEUP>(a, ash, b64, b16, args, s);
-    case 192: return launch_gemm_t<192, GATEUP>(a, ash, b64, b16, args, s);
-    case 256: return launch_gemm_t<256, GATEUP>(a, ash, b64, b16, args, s);
-    default: return cudaErrorInvalidValue;
+    case 16: return launch_gemm_t<16, MODE>(a, ash, b64, b16, args, s);
+    case 32: return launch_gemm_t<32, MODE>(a, ash, b64, b16, args, s);
+    case 64: return launch_gemm_t<64, MODE>(a, ash, b64, b16, args, s);
+    default:
+      if constexpr (MODE == kModeGateUpPartial) return cudaErrorInvalidValue;  // decode tiles only
+      switch (BN) {
+        case 128: return launch_gemm_t<128, MODE>(a, ash, b64, b16, args, s);
+        case 192: return launch_gemm_t<192, MODE>(a, ash, b64, b16, args, s);
+        case 256: return launch_gemm_t<256, MODE>(a, ash, b64, b16, args, s);
+        default: return cudaErrorInvalidValue;
+      }
   }
 }
 }  // namespace
 
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
                                const CUtensorMap& acts64, const CUtensorMap& acts16,
-                               const GemmArgs& a, cudaStream_t s) {
-  return launch_by_bn<true>(p.BN, w13, w13s, acts64, acts16, a, s);
+                               const GemmArgs& a, bool partial, cudaStream_t s) {
+  if (partial) return launch_by_bn<kModeGateUpPartial>(p.BN, w13, w13s, acts64, acts16, a, s);
+  return launch_by_bn<kModeSwiGLU>(p.BN, w13, w13s, acts64, acts16, a, s);
 }
 
 cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
                              const CUtensorMap& acts64, const CUtensorMap& acts16,
                              const GemmArgs& a, cudaStream_t s) {
-  return launch_by_bn<false>(p.BN, w2, w2s, acts64, acts16, a, s);
+  return launch_by_bn<kModeDown>(p.BN, w2, w2s, acts64, acts16, a, s);
 }
 
 }  // namespace moe

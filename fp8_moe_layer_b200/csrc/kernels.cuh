@@ -24,11 +24,19 @@ struct Plan {
   int BN;            // token tile of the grouped GEMMs (max MMA N; a tile uses its valid rows)
   int r_splits, r_chunks_per_split;           // router: split of d into 32-wide chunks
   int g1_kb, g1_m_tiles;                      // gate/up GEMM: K blocks (d/128), 64-row tiles
+  int g1_splits, g1_kb_per_split;             // gate/up K split (decode); 1 = SwiGLU epilogue
   int g2_kb, g2_m_tiles, g2_splits, g2_kb_per_split;  // down GEMM
   size_t off_status, off_part, off_ids, off_w, off_offsets, off_tiles, off_perm, off_inv, off_pscr;
   size_t off_xq, off_xs, off_xqp, off_xsp, off_amax, off_act, off_aq, off_s2, off_o, off_planes;
+  size_t off_hpart;
   size_t bytes;
 };
+
+// Grouped GEMM variants: gate/up with the SwiGLU epilogue (act + row max), down projection, and
+// gate/up split over K (scaled partial sums; SwiGLU and the requantisation follow in a row kernel).
+constexpr int kModeSwiGLU = 0;
+constexpr int kModeDown = 1;
+constexpr int kModeGateUpPartial = 2;
 
 // Arguments of one grouped GEMM launch (tile decode + epilogue).
 struct GemmArgs {
@@ -85,7 +93,11 @@ cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, con
 // acts64 / acts16: the routed-row activations with 64-row and 16-row TMA boxes
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
                                const CUtensorMap& acts64, const CUtensorMap& acts16,
-                               const GemmArgs& a, cudaStream_t s);
+                               const GemmArgs& a, bool partial, cudaStream_t s);
+// K-split gate/up: h[s][r][2F] partials -> act = silu(gate) * up, row amax, FP8 codes and scales
+cudaError_t launch_swiglu_requant(const Plan& p, const float* h, int splits, size_t split_stride,
+                                  const int32_t* total_rows, uint8_t* aq, float* s2,
+                                  cudaStream_t s);
 cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
                              const CUtensorMap& acts64, const CUtensorMap& acts16,
                              const GemmArgs& a, cudaStream_t s);

@@ -85,10 +85,19 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
 
   p->g1_kb = (int)ceil_div(d, kBK);
   p->g1_m_tiles = (int)ceil_div(F, 64);
+  // gate/up: split K (partial sums + a row kernel for SwiGLU) when the tiles would leave the last
+  // wave of SMs mostly idle; only for decode-sized token tiles
+  p->g1_splits = 1;
+  p->g1_kb_per_split = p->g1_kb;
   p->g2_kb = (int)ceil_div(F, kBK);
   p->g2_m_tiles = (int)ceil_div(d, 128);
   const int64_t est_ntiles = std::max<int64_t>(active, ceil_div(routed, BN)) +
                              (p->shared ? ceil_div(T, BN) : 0);
+  if (BN <= 64) {
+    const int s1 = choose_splits(est_ntiles * p->g1_m_tiles, p->g1_kb);
+    p->g1_kb_per_split = (int)ceil_div(p->g1_kb, s1);
+    p->g1_splits = (int)ceil_div(p->g1_kb, p->g1_kb_per_split);
+  }
   int s2 = choose_splits(est_ntiles * p->g2_m_tiles, p->g2_kb);
   p->g2_kb_per_split = (int)ceil_div(p->g2_kb, s2);
   p->g2_splits = (int)ceil_div(p->g2_kb, p->g2_kb_per_split);   // every split non-empty
@@ -114,6 +123,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
   p->off_s2 = take(sizeof(float) * (size_t)p->Rpad);
   p->off_o = take(sizeof(float) * (size_t)p->g2_splits * p->Rpad * d);
   p->off_planes = take(router_uses_mma(E, T) ? 3 * sizeof(uint16_t) * (size_t)E * d : 0);
+  p->off_hpart = take(p->g1_splits > 1 ? sizeof(float) * p->g1_splits * (size_t)p->Rcap * 2 * F : 0);
   p->bytes = off;
   return MOE_OK;
 }
@@ -212,7 +222,7 @@ static int check_device() {
 
 struct Ws {
   int* status;
-  float *part, *w, *xs, *xsp, *act, *s2, *o;
+  float *part, *w, *xs, *xsp, *act, *s2, *o, *hpart;
   uint16_t* planes;
   int32_t *ids, *offsets, *tiles, *perm, *inv, *pscr;
   uint8_t *xq, *xqp, *aq;
@@ -241,6 +251,7 @@ static Ws carve(const Plan& p, void* ws) {
   w.s2 = reinterpret_cast<float*>(b + p.off_s2);
   w.o = reinterpret_cast<float*>(b + p.off_o);
   w.planes = reinterpret_cast<uint16_t*>(b + p.off_planes);
+  w.hpart = reinterpret_cast<float*>(b + p.off_hpart);
   return w;
 }
 
@@ -324,11 +335,24 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g1.out_split_stride = 0;
   g1.row_amax = w.amax;
   g1.status = w.status;
+  const bool split1 = p.g1_splits > 1;
+  if (split1) {
+    g1.splits = p.g1_splits;
+    g1.kb_per_split = p.g1_kb_per_split;
+    g1.out = w.hpart;
+    g1.out_ld = 2 * p.F;
+    g1.out_split_stride = (size_t)p.Rcap * 2 * p.F;
+    g1.row_amax = nullptr;
+  }
   record(4);
-  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mxq64, mxq16, g1, s));
+  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mxq64, mxq16, g1, split1, s));
 
   record(5);
-  MOE_CUDA(launch_requant(p, w.act, w.amax, total_rows, w.aq, w.s2, s));
+  if (split1)
+    MOE_CUDA(launch_swiglu_requant(p, w.hpart, p.g1_splits, g1.out_split_stride, total_rows, w.aq,
+                                   w.s2, s));
+  else
+    MOE_CUDA(launch_requant(p, w.act, w.amax, total_rows, w.aq, w.s2, s));
 
   GemmArgs g2 = g1;
   g2.m_tiles = p.g2_m_tiles;

@@ -267,6 +267,8 @@ __global__ void __launch_bounds__(256) route_block_kernel(
     int T, int d, int E, int k, const int32_t* __restrict__ k_per_token, int k_max,
     int32_t* __restrict__ ids, float* __restrict__ wout, uint8_t* __restrict__ xq,
     float* __restrict__ xs, int do_quant, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
   constexpr int kChunks = 4;                      // d <= 256 * 8 * kChunks = 8192
   __shared__ float part[8][EP];
   __shared__ float red[8];
