@@ -43,17 +43,18 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
 
 // K-split gate/up: per routed row, gate[f] = sum_s h[s][r][f], up[f] = sum_s h[s][r][F + f]
 // (split order fixed), act = silu(gate) * up, s2 = amax|act| / 448 (IEEE fp32; 1 if 0),
-// aq = e4m3(act / s2). One block per row; act is recomputed in the second pass instead of stored.
-__global__ void __launch_bounds__(256) swiglu_requant_kernel(
+// aq = e4m3(act / s2). One block (up to 1024 threads) per row; act is recomputed in the second
+// pass instead of stored.
+__global__ void __launch_bounds__(1024) swiglu_requant_kernel(
     const float* __restrict__ h, int splits, size_t split_stride,
     const int32_t* __restrict__ total_rows, int64_t rcap, int F, uint8_t* __restrict__ aq,
     float* __restrict__ s2) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  __shared__ float red[8];
+  __shared__ float red[32];
   const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
   const int nv = F / 4;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     auto act4 = [&](int i) {
       const float4* g4 = reinterpret_cast<const float4*>(h + (size_t)r * 2 * F);
@@ -77,8 +78,7 @@ __global__ void __launch_bounds__(256) swiglu_requant_kernel(
     if (lane == 0) red[warp] = amax;
     __syncthreads();
     float am = red[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) am = fmaxf(am, red[w]);
+    for (int w = 1; w < nwarps; ++w) am = fmaxf(am, red[w]);
     const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
     if (threadIdx.x == 0) s2[r] = sc;
     uint32_t* dst = reinterpret_cast<uint32_t*>(aq + (size_t)r * F);
@@ -189,7 +189,9 @@ cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax
 cudaError_t launch_swiglu_requant(const Plan& p, const float* h, int splits, size_t split_stride,
                                   const int32_t* total_rows, uint8_t* aq, float* s2,
                                   cudaStream_t s) {
-  launch_pdl(swiglu_requant_kernel, dim3(row_grid(p.Rcap)), dim3(256), 0, s, h, splits,
+  // few long rows at decode: up to 1024 threads per row (one float4 of F per thread)
+  const int threads = std::min(1024, std::max(128, ((p.F / 4 + 31) / 32) * 32));
+  launch_pdl(swiglu_requant_kernel, dim3(row_grid(p.Rcap)), dim3(threads), 0, s, h, splits,
              split_stride, total_rows, p.Rcap, p.F, aq, s2);
   return cudaGetLastError();
 }
