@@ -32,14 +32,18 @@
 
 namespace moe {
 
-template <int BN, int MODE>
+template <int BN, int MODE, bool PAIR>
 struct GemmCfg {
-  static constexpr int BM = 128;
+  static constexpr int BM = 128;                           // weight rows held by one CTA
+  static constexpr int BROWS = PAIR ? BN / 2 : BN;         // token rows held by one CTA
+  static constexpr int ROUND = PAIR ? 32 : 16;             // MMA N granule (halves of 16 rows)
   static constexpr int A_BYTES = BM * kBK;
-  static constexpr int B_BYTES = BN * kBK;
+  static constexpr int B_BYTES = BROWS * kBK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int XCHG_LD = 33;                       // padded row of the exchange buffer
-  static constexpr int XCHG_BYTES = MODE == kModeSwiGLU ? 128 * XCHG_LD * 4 : 0;
+  // SwiGLU: gate/up exchange; down GEMM with prefill tiles: per-warp transpose for 16-byte stores
+  static constexpr bool DOWN_T = MODE == kModeDown && BN >= 128;
+  static constexpr int XCHG_BYTES = (MODE == kModeSwiGLU || DOWN_T) ? 128 * XCHG_LD * 4 : 0;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_MAX = 232448;                  // 227 KB per block
   // group offsets and tile prefix of up to kMaxExperts + 1 groups, cached in shared memory
@@ -55,6 +59,7 @@ struct GemmCfg {
   static_assert(STAGES >= 3, "pipeline too shallow");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128");
   static_assert(BN % CW == 0, "epilogue chunks");
+  static_assert(!PAIR || (BN >= 64 && MODE != kModeGateUpPartial), "pair tiles: prefill shapes");
 };
 
 // The tile list, read from shared-memory copies of the group offsets and the tile prefix (a tile
@@ -85,15 +90,15 @@ __device__ __forceinline__ void decode_tile(const TileTable& tt, int tile, int& 
   m = rest / tt.splits;
 }
 
-// Valid token rows of the tile starting at row0 of group g, rounded up to a multiple of 16.
-template <int BN>
-__device__ __forceinline__ int tile_rows16(const TileTable& tt, int g, int row0) {
+// Valid token rows of the tile starting at row0 of group g, rounded up to a multiple of ROUND.
+template <int BN, int ROUND>
+__device__ __forceinline__ int tile_rows_rounded(const TileTable& tt, int g, int row0) {
   const int rows = min(BN, tt.off[g + 1] - row0);
-  return (rows + 15) & ~15;
+  return (rows + ROUND - 1) / ROUND * ROUND;
 }
 
 
-template <int BN, int MODE>
+template <int BN, int MODE, bool PAIR>
 __global__ void __launch_bounds__(256, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_a_shared,
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(256, 1)
                         const __grid_constant__ CUtensorMap map_b16, const GemmArgs args) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  using C = GemmCfg<BN, MODE>;
+  using C = GemmCfg<BN, MODE, PAIR>;
   constexpr bool kGateUp = MODE != kModeDown;     // A tile = 64 gate rows + the 64 up rows
   constexpr int kWhere = kGateUp ? kWhereGemm1 : kWhereGemm2;
   extern __shared__ uint8_t smem_raw[];
@@ -116,15 +121,23 @@ __global__ void __launch_bounds__(256, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total_tiles = args.m_tiles * args.splits * args.tile_prefix[args.G];
-  if (static_cast<int>(blockIdx.x) >= total_tiles) return;
+  // A pair (2-CTA cluster) works on one tile of 256 weight rows: CTA rank r holds weight m-tile
+  // 2 mu + r and half of the token rows; the even CTA issues the MMAs. Both CTAs of a pair see
+  // the same tile sequence, so they leave (or stay) together.
+  const uint32_t crank = PAIR ? cluster_rank() : 0u;
+  const bool leader = crank == 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nunits = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  const int m_units = PAIR ? (args.m_tiles + 1) / 2 : args.m_tiles;
+  const int total_tiles = m_units * args.splits * args.tile_prefix[args.G];
+  if (unit >= total_tiles) return;
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
   int* s_tp = s_off + (kMaxExperts + 2);
   for (int i = threadIdx.x; i <= args.G; i += blockDim.x) {
     s_off[i] = args.group_offsets[i];
     s_tp[i] = args.tile_prefix[i];
   }
-  const TileTable tt{s_off, s_tp, args.G, args.m_tiles * args.splits, args.splits};
+  const TileTable tt{s_off, s_tp, args.G, m_units * args.splits, args.splits};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -133,19 +146,28 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], PAIR ? 8 : 4);     // the epilogue warps of both CTAs of a pair
     }
     mbar_init(drain, 1);
     fence_mbarrier_init();
   }
   if (warp == 2) {
-    tmem_alloc(tmem_slot, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();    // both CTAs' barriers initialised before any remote use
+  else __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // shared::cluster addresses of the even CTA's barriers (pair loads, commits and arrivals)
+  const uint32_t full_l = PAIR ? cluster_addr(full, 0) : 0u;
+  const uint32_t tempty_l = PAIR ? cluster_addr(tempty, 0) : 0u;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -159,39 +181,60 @@ __global__ void __launch_bounds__(256, 1)
       int stage = 0, issued = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-        int g, m, n, s;
-        decode_tile(tt, tile, g, m, n, s);
+      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
+        int g, mu, n, s;
+        decode_tile(tt, tile, g, mu, n, s);
+        const int m = PAIR ? 2 * mu + static_cast<int>(crank) : mu;
         const int row0 = tt.off[g] + n * BN;
-        const int rows16 = tile_rows16<BN>(tt, g, row0);   // valid token rows, rounded to 16
-        const uint32_t stage_bytes = C::A_BYTES + rows16 * kBK;
+        const int rowsN = tile_rows_rounded<BN, C::ROUND>(tt, g, row0);   // the MMA's N
+        const int myrows = PAIR ? rowsN / 2 : rowsN;       // token rows this CTA loads
+        const int myrow0 = row0 + static_cast<int>(crank) * myrows;
+        // bytes that complete the (even CTA's) full barrier: both CTAs' loads for a pair
+        const uint32_t stage_bytes = (PAIR ? 2 : 1) * C::A_BYTES + rowsN * kBK;
         const int kb0 = s * args.kb_per_split;
         const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
         const bool sh = g >= args.E_routed;
         const CUtensorMap* ma = sh ? &map_a_shared : &map_a;
         const int ga = sh ? 0 : g;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u)) {
+          const bool got = PAIR ? mbar_wait_cluster(&empty[stage], phase ^ 1u)
+                                : mbar_wait(&empty[stage], phase ^ 1u);
+          if (!got) {
             report(args.status, kStatusDeviceTimeout, kWhere, 1);
             ok = false;
             break;
           }
           uint8_t* sa = stages + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], stage_bytes);
-          if (kGateUp) {
-            tma_load_4d(sa, ma, &full[stage], kb * kBK, m * 64, 0, ga, pol_w);
-            tma_load_4d(sa + C::A_BYTES / 2, ma, &full[stage], kb * kBK, m * 64, 1, ga, pol_w);
-          } else {
-            tma_load_3d(sa, ma, &full[stage], kb * kBK, m * 128, ga, pol_w);
-          }
-          // only the tile's valid token rows: 64-row boxes, then 16-row boxes
           uint8_t* sb = sa + C::A_BYTES;
-          int r = 0;
-          if constexpr (BN >= 64)
-            for (; r + 64 <= rows16; r += 64)
-              tma_load_2d(sb + r * kBK, &map_b64, &full[stage], kb * kBK, row0 + r, pol_x);
-          for (; r < rows16; r += 16)
-            tma_load_2d(sb + r * kBK, &map_b16, &full[stage], kb * kBK, row0 + r, pol_x);
+          if (leader) mbar_arrive_expect_tx(&full[stage], stage_bytes);
+          if constexpr (PAIR) {
+            const uint32_t fb = full_l + 8u * stage;
+            if (kGateUp) {
+              tma_load_4d_pair(sa, ma, fb, kb * kBK, m * 64, 0, ga, pol_w);
+              tma_load_4d_pair(sa + C::A_BYTES / 2, ma, fb, kb * kBK, m * 64, 1, ga, pol_w);
+            } else {
+              tma_load_3d_pair(sa, ma, fb, kb * kBK, m * 128, ga, pol_w);
+            }
+            int r = 0;
+            for (; r + 64 <= myrows; r += 64)
+              tma_load_2d_pair(sb + r * kBK, &map_b64, fb, kb * kBK, myrow0 + r, pol_x);
+            for (; r < myrows; r += 16)
+              tma_load_2d_pair(sb + r * kBK, &map_b16, fb, kb * kBK, myrow0 + r, pol_x);
+          } else {
+            if (kGateUp) {
+              tma_load_4d(sa, ma, &full[stage], kb * kBK, m * 64, 0, ga, pol_w);
+              tma_load_4d(sa + C::A_BYTES / 2, ma, &full[stage], kb * kBK, m * 64, 1, ga, pol_w);
+            } else {
+              tma_load_3d(sa, ma, &full[stage], kb * kBK, m * 128, ga, pol_w);
+            }
+            // only the tile's valid token rows: 64-row boxes, then 16-row boxes
+            int r = 0;
+            if constexpr (BN >= 64)
+              for (; r + 64 <= myrows; r += 64)
+                tma_load_2d(sb + r * kBK, &map_b64, &full[stage], kb * kBK, myrow0 + r, pol_x);
+            for (; r < myrows; r += 16)
+              tma_load_2d(sb + r * kBK, &map_b16, &full[stage], kb * kBK, myrow0 + r, pol_x);
+          }
           ++issued;
           if (++stage == C::STAGES) {
             stage = 0;
@@ -199,8 +242,10 @@ __global__ void __launch_bounds__(256, 1)
           }
         }
       }
-      // Drain: the most recent load of every stage must have landed before the CTA exits.
-      const int outstanding = min(issued, C::STAGES);
+      // Drain: the most recent load of every stage must have landed before the CTA exits. (In
+      // a pair the even CTA's full barriers count both CTAs' bytes; the odd CTA relies on the
+      // final cluster barrier, which the even CTA reaches only after this drain.)
+      const int outstanding = leader ? min(issued, C::STAGES) : 0;
       for (int i = 0; i < outstanding; ++i) {
         int st = stage - 1 - i;
         uint32_t ph = phase;
@@ -212,22 +257,30 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (one thread)
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (one thread; in a
+    // pair the even CTA's, for both CTAs)
+    if (lane == 0 && leader) {
       int stage = 0, it = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
-        int g, m, n, s;
-        decode_tile(tt, tile, g, m, n, s);
+      const uint32_t empty_l = PAIR ? cluster_addr(empty, 0) : 0u;
+      const uint32_t empty_p = PAIR ? cluster_addr(empty, 1) : 0u;
+      const uint32_t tfull_l = PAIR ? cluster_addr(tfull, 0) : 0u;
+      const uint32_t tfull_p = PAIR ? cluster_addr(tfull, 1) : 0u;
+      for (int tile = unit; ok && tile < total_tiles; tile += nunits, ++it) {
+        int g, mu, n, s;
+        decode_tile(tt, tile, g, mu, n, s);
         const int kb0 = s * args.kb_per_split;
         const int kb1 = min(args.num_kb, kb0 + args.kb_per_split);
-        // MMA N = the tile's valid rows rounded up to 16 (M = 128 takes N = 16 .. 256 by 16)
-        const uint32_t idesc =
-            idesc_e4m3_f32(128, tile_rows16<BN>(tt, g, tt.off[g] + n * BN));
+        // MMA N = the tile's valid rows rounded up (M = 128 takes N = 16 .. 256 by 16; the pair's
+        // M = 256 the same, here by 32 so that each CTA's half is whole 16-row boxes)
+        const uint32_t idesc = idesc_e4m3_f32(
+            PAIR ? 256 : 128, tile_rows_rounded<BN, C::ROUND>(tt, g, tt.off[g] + n * BN));
         const int ab = it & 1;
         const uint32_t aph = (it >> 1) & 1;
-        if (!mbar_wait(&tempty[ab], aph ^ 1u)) {
+        const bool freed = PAIR ? mbar_wait_cluster(&tempty[ab], aph ^ 1u)
+                                : mbar_wait(&tempty[ab], aph ^ 1u);
+        if (!freed) {
           report(args.status, kStatusDeviceTimeout, kWhere, 2);
           ok = false;
           break;
@@ -245,18 +298,37 @@ __global__ void __launch_bounds__(256, 1)
           const uint64_t adesc = smem_desc_sw128(sa);
           const uint64_t bdesc = smem_desc_sw128(sa + C::A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 32; ++kk)   // K = 32 e4m3 (32 bytes) per instruction
-            mma_e4m3(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                     (kb > kb0 || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[stage]);               // frees the stage when these MMAs finish
+          for (int kk = 0; kk < kBK / 32; ++kk) {  // K = 32 e4m3 (32 bytes) per instruction
+            if constexpr (PAIR)
+              mma_e4m3_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                            (kb > kb0 || kk > 0) ? 1u : 0u);
+            else
+              mma_e4m3(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                       (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          // frees the stage (in both CTAs of a pair) when these MMAs finish
+          if constexpr (PAIR) {
+            mma_commit_pair(empty_l + 8u * stage);
+            mma_commit_pair(empty_p + 8u * stage);
+          } else {
+            mma_commit(&empty[stage]);
+          }
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) mma_commit(&tfull[ab]);            // accumulator ready for the epilogue
+        if (ok) {                                  // accumulator ready for the epilogue(s)
+          if constexpr (PAIR) {
+            mma_commit_pair(tfull_l + 8u * ab);
+            mma_commit_pair(tfull_p + 8u * ab);
+          } else {
+            mma_commit(&tfull[ab]);
+          }
+        }
       }
-      mma_commit(drain);
+      if constexpr (PAIR) mma_commit_pair(cluster_addr(drain, 0));
+      else mma_commit(drain);
       mbar_wait(drain, 0);
     }
   } else if (warp >= 4) {
@@ -266,21 +338,51 @@ __global__ void __launch_bounds__(256, 1)
     const int q = warp & 3;
     bool bad = false;
     int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      int g, m, n, s;
-      decode_tile(tt, tile, g, m, n, s);
+    for (int tile = unit; tile < total_tiles; tile += nunits, ++it) {
+      int g, mu, n, s;
+      decode_tile(tt, tile, g, mu, n, s);
+      const int m = PAIR ? 2 * mu + static_cast<int>(crank) : mu;
       const int ab = it & 1;
       const uint32_t aph = (it >> 1) & 1;
+      // this lane's row scales (token column CW u + lane of every column chunk u) and weight
+      // scale, loaded before the accumulator wait so that their latency hides behind it
+      constexpr int kRsRegs = BN / C::CW;
+      float rs[kRsRegs];
+      {
+        const int row0p = tt.off[g] + n * BN;
+        const int nv = min(BN, tt.off[g + 1] - row0p);
+#pragma unroll
+        for (int u = 0; u < kRsRegs; ++u) {
+          const int c = u * C::CW + lane;
+          rs[u] = (c < nv && (C::CW == 32 || lane < C::CW)) ? args.row_scale[row0p + c] : 0.f;
+        }
+      }
+      // output channel of this lane: the weight row of TMEM lane 32 q + lane
+      int ch;
+      bool valid;
+      float wsv;
+      {
+        const bool sh = g >= args.E_routed;
+        const float* wsc = sh ? args.w_scale_shared : args.w_scale + (size_t)g * args.w_scale_ld;
+        if constexpr (MODE == kModeDown) {
+          ch = m * 128 + 32 * q + lane;                      // down: output channel i
+          valid = ch < args.M_valid;
+          wsv = valid ? wsc[ch] : 0.f;
+        } else {
+          const int frow = m * 64 + 32 * (q & 1) + lane;    // gate (q < 2) / up (q >= 2) row
+          valid = frow < args.M_valid;
+          ch = (q >> 1) * args.M_valid + frow;               // its column of [gate | up]
+          wsv = valid ? wsc[ch] : 0.f;
+        }
+      }
       if (!bad) {
-        const bool ok = mbar_wait(&tfull[ab], aph);
+        const bool ok = PAIR ? mbar_wait_cluster(&tfull[ab], aph) : mbar_wait(&tfull[ab], aph);
         bad = __any_sync(0xffffffffu, !ok);         // warp-uniform: TMEM loads are .sync.aligned
         if (bad && lane == 0) report(args.status, kStatusDeviceTimeout, kWhere, 5);
       }
       tc_fence_after_sync();
       const int row0 = tt.off[g] + n * BN;
       const int nvalid = min(BN, tt.off[g + 1] - row0);
-      const bool sh = g >= args.E_routed;
-      const float* wsc = sh ? args.w_scale_shared : args.w_scale + (size_t)g * args.w_scale_ld;
       const uint32_t tbase = tmem_base + ab * BN + (static_cast<uint32_t>(32 * q) << 16);
       if constexpr (MODE == kModeSwiGLU) {
         // TMEM lane 32q+i holds gate row (q<2) or up row (q>=2) 32*(q&1)+i of this 64-row half
@@ -288,10 +390,12 @@ __global__ void __launch_bounds__(256, 1)
         // Step 2: thread (q, lane) takes token column `lane` and the 16 features 16q .. 16q+15:
         // SwiGLU, one 64-byte store, and the in-thread max |act| for the row amax.
         constexpr int CW = C::CW;
-        const int frow = m * 64 + 32 * (q & 1) + lane;
-        const float wsv = frow < args.M_valid ? wsc[(q >> 1) * args.M_valid + frow] : 0.f;
         const int f0 = m * 64 + 16 * q;                // this thread's first feature
-        for (int c0 = 0; c0 < nvalid; c0 += CW) {
+        for (int c0 = 0, j = 0; c0 < nvalid; c0 += CW, ++j) {
+          float rsv = 0.f;
+#pragma unroll
+          for (int u = 0; u < kRsRegs; ++u)
+            if (u == j) rsv = rs[u];
           if (!bad) {
             uint32_t r[CW];
             tmem_ld16(tbase + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
@@ -305,14 +409,14 @@ __global__ void __launch_bounds__(256, 1)
           named_bar_sync(1, 128);
           const int nn = c0 + lane;
           if (!bad && lane < CW && nn < nvalid && f0 < args.M_valid) {
-            const float rs = args.row_scale[row0 + nn];
+            const float rs = rsv;
             float act[16];
             float amax = 0.f;
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
-              const int j = 16 * q + jj;
-              const float gv = xchg[j * C::XCHG_LD + lane] * rs;
-              const float uv = xchg[(64 + j) * C::XCHG_LD + lane] * rs;
+              const int jf = 16 * q + jj;
+              const float gv = xchg[jf * C::XCHG_LD + lane] * rs;
+              const float uv = xchg[(64 + jf) * C::XCHG_LD + lane] * rs;
               act[jj] = silu(gv) * uv;
               amax = fmaxf(amax, fabsf(act[jj]));
             }
@@ -324,91 +428,145 @@ __global__ void __launch_bounds__(256, 1)
           }
           named_bar_sync(1, 128);
         }
-      } else if constexpr (MODE == kModeGateUpPartial) {
-        // K-split gate/up: scaled partial sums of gate (columns [0, F)) and up ([F, 2F)) rows
-        const int half = q >> 1;
-        const int frow = m * 64 + 32 * (q & 1) + lane;
-        const bool valid_row = frow < args.M_valid;
-        const float wsv = valid_row ? wsc[half * args.M_valid + frow] : 0.f;
-        const int col = half * args.M_valid + frow;
-        float* outp = args.out + (size_t)s * args.out_split_stride;
-        for (int c0 = 0; !bad && c0 < nvalid; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(tbase + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int nn = c0 + c;
-            if (nn < nvalid && valid_row)
-              outp[(size_t)(row0 + nn) * args.out_ld + col] =
-                  __uint_as_float(r[c]) * args.row_scale[row0 + nn] * wsv;
-          }
-        }
       } else {
-        const int i = m * 128 + 32 * q + lane;         // output channel
-        const float wsv = i < args.M_valid ? wsc[i] : 0.f;
-        float* outp = args.out + (size_t)s * args.out_split_stride;
-        for (int c0 = 0; !bad && c0 < nvalid; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(tbase + c0, r);
-          tmem_wait_ld();
+        // Down GEMM (output channel i = TMEM lane) or K-split gate/up (gate column frow of
+        // [0, F), up column F + frow). Lane l holds the row scales of token columns
+        // c0 + l of every 32-column chunk (one coalesced load per chunk, issued above before
+        // the accumulator wait); a shuffle hands column c's scale to the whole warp.
+        constexpr int CW = C::CW;
+        float* outp = args.out + (size_t)s * args.out_split_stride + (size_t)row0 * args.out_ld + ch;
+#pragma unroll 1
+        for (int j = 0; !bad && j * CW < nvalid; ++j) {
+          const int c0 = j * CW;
+          uint32_t r[CW];
+          tmem_ld16(tbase + c0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+          if constexpr (CW == 32)
+            tmem_ld16(tbase + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+          float rsv = 0.f;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int nn = c0 + c;
-            if (nn < nvalid && i < args.M_valid)
-              outp[(size_t)(row0 + nn) * args.out_ld + i] =
-                  __uint_as_float(r[c]) * args.row_scale[row0 + nn] * wsv;
+          for (int u = 0; u < kRsRegs; ++u)
+            if (u == j) rsv = rs[u];
+          tmem_wait_ld();
+          const int ncol = min(CW, nvalid - c0);
+          float* dst = outp + (size_t)c0 * args.out_ld;
+          float v[CW];
+#pragma unroll
+          for (int c = 0; c < CW; ++c)
+            v[c] = __uint_as_float(r[c]) * __shfl_sync(0xffffffffu, rsv, c) * wsv;
+          if constexpr (C::DOWN_T) {
+            // Through this warp's 32 x 33 block of shared memory: lane l then writes channels
+            // 4 (l % 8) .. +3 of token 4 i + l / 8 as one 16-byte store (a quarter of the store
+            // instructions of one 4-byte store per token; in this kernel the store instruction
+            // count, not the bytes, sets the pace of the epilogue).
+            float* tr = xchg + 32 * q * C::XCHG_LD;
+#pragma unroll
+            for (int c = 0; c < CW; ++c) tr[c * C::XCHG_LD + lane] = v[c];
+            __syncwarp();
+            const int chq = m * 128 + 32 * q, cc = 4 * (lane & 7);
+            float* base = args.out + (size_t)s * args.out_split_stride +
+                          (size_t)(row0 + c0) * args.out_ld + chq + cc;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int c = 4 * i + (lane >> 3);
+              if (c < ncol && chq + cc < args.M_valid) {
+                const float* t4 = tr + c * C::XCHG_LD + cc;
+                *reinterpret_cast<float4*>(base + (size_t)c * args.out_ld) =
+                    make_float4(t4[0], t4[1], t4[2], t4[3]);
+              }
+            }
+            __syncwarp();
+          } else if (valid) {
+#pragma unroll
+            for (int c = 0; c < CW; ++c)
+              if (c < ncol) dst[(size_t)c * args.out_ld] = v[c];
           }
         }
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (!bad && lane == 0) mbar_arrive(&tempty[ab]);
+      if (!bad && lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(tempty_l + 8u * ab);   // the even CTA's barrier
+        else mbar_arrive(&tempty[ab]);
+      }
     }
   }
 
   tc_fence_before_sync();
-  __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();   // no CTA leaves while its pair still uses its memory
+  else __syncthreads();
   if (warp == 2) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
 namespace {
-template <int BN, int MODE>
+template <int BN, int MODE, bool PAIR>
 cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& ash, const CUtensorMap& b64,
                           const CUtensorMap& b16, const GemmArgs& args, cudaStream_t s) {
-  using C = GemmCfg<BN, MODE>;
-  static bool attr_done[64] = {};
+  using C = GemmCfg<BN, MODE, PAIR>;
+  static int grid_cache[64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 64 && !attr_done[dev]) {
-    err = cudaFuncSetAttribute(grouped_gemm_kernel<BN, MODE>,
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (!grid_cache[dev]) {
+    err = cudaFuncSetAttribute(grouped_gemm_kernel<BN, MODE, PAIR>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (err != cudaSuccess) return err;
-    attr_done[dev] = true;
+    int grid = num_sms();
+    if (PAIR) {
+      // persistent pairs: as many 2-CTA clusters as can be resident at once
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(num_sms());
+      cfg.blockDim = dim3(256);
+      cfg.dynamicSmemBytes = C::SMEM;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      err = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_kernel<BN, MODE, PAIR>, &cfg);
+      if (err != cudaSuccess) return err;
+      if (clusters < 1) return cudaErrorInvalidConfiguration;
+      grid = 2 * std::min(clusters, num_sms() / 2);
+    }
+    grid_cache[dev] = grid;
   }
-  launch_pdl(grouped_gemm_kernel<BN, MODE>, dim3(num_sms()), dim3(256), C::SMEM, s, a, ash, b64, b16, args);
+  launch_pdl_cluster(grouped_gemm_kernel<BN, MODE, PAIR>, dim3(grid_cache[dev]), dim3(256), C::SMEM,
+                     PAIR ? 2 : 1, s, a, ash, b64, b16, args);
   return cudaGetLastError();
 }
 
 template <int MODE>
-cudaError_t launch_by_bn(int BN, const CUtensorMap& a, const CUtensorMap& ash,
+cudaError_t launch_by_bn(int BN, bool pair, const CUtensorMap& a, const CUtensorMap& ash,
                          const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& args,
                          cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_gemm_t<16, MODE>(a, ash, b64, b16, args, s);
-    case 32: return launch_gemm_t<32, MODE>(a, ash, b64, b16, args, s);
-    case 64: return launch_gemm_t<64, MODE>(a, ash, b64, b16, args, s);
+    case 16: return launch_gemm_t<16, MODE, false>(a, ash, b64, b16, args, s);
+    case 32: return launch_gemm_t<32, MODE, false>(a, ash, b64, b16, args, s);
+    case 64: return launch_gemm_t<64, MODE, false>(a, ash, b64, b16, args, s);
     default:
       if constexpr (MODE == kModeGateUpPartial) return cudaErrorInvalidValue;  // decode tiles only
-      switch (BN) {
-        case 128: return launch_gemm_t<128, MODE>(a, ash, b64, b16, args, s);
-        case 192: return launch_gemm_t<192, MODE>(a, ash, b64, b16, args, s);
-        case 256: return launch_gemm_t<256, MODE>(a, ash, b64, b16, args, s);
-        default: return cudaErrorInvalidValue;
+      else {
+        if (pair) {
+          switch (BN) {
+            case 128: return launch_gemm_t<128, MODE, true>(a, ash, b64, b16, args, s);
+            case 192: return launch_gemm_t<192, MODE, true>(a, ash, b64, b16, args, s);
+            case 256: return launch_gemm_t<256, MODE, true>(a, ash, b64, b16, args, s);
+            default: return cudaErrorInvalidValue;
+          }
+        }
+        switch (BN) {
+          case 128: return launch_gemm_t<128, MODE, false>(a, ash, b64, b16, args, s);
+          case 192: return launch_gemm_t<192, MODE, false>(a, ash, b64, b16, args, s);
+          case 256: return launch_gemm_t<256, MODE, false>(a, ash, b64, b16, args, s);
+          default: return cudaErrorInvalidValue;
+        }
       }
   }
 }
@@ -417,14 +575,14 @@ cudaError_t launch_by_bn(int BN, const CUtensorMap& a, const CUtensorMap& ash,
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
                                const CUtensorMap& acts64, const CUtensorMap& acts16,
                                const GemmArgs& a, bool partial, cudaStream_t s) {
-  if (partial) return launch_by_bn<kModeGateUpPartial>(p.BN, w13, w13s, acts64, acts16, a, s);
-  return launch_by_bn<kModeSwiGLU>(p.BN, w13, w13s, acts64, acts16, a, s);
+  if (partial) return launch_by_bn<kModeGateUpPartial>(p.BN, false, w13, w13s, acts64, acts16, a, s);
+  return launch_by_bn<kModeSwiGLU>(p.BN, p.pair1, w13, w13s, acts64, acts16, a, s);
 }
 
 cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
                              const CUtensorMap& acts64, const CUtensorMap& acts16,
                              const GemmArgs& a, cudaStream_t s) {
-  return launch_by_bn<kModeDown>(p.BN, w2, w2s, acts64, acts16, a, s);
+  return launch_by_bn<kModeDown>(p.BN, p.pair2, w2, w2s, acts64, acts16, a, s);
 }
 
 }  // namespace moe

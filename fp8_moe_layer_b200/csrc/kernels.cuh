@@ -22,6 +22,7 @@ struct Plan {
   int64_t Rcap;      // routed-row capacity: T*k_max (+T shared rows)
   int64_t Rpad;      // rows allocated for row-indexed buffers (>= Rcap, >= 256)
   int BN;            // token tile of the grouped GEMMs (max MMA N; a tile uses its valid rows)
+  bool pair1, pair2; // gate/up, down GEMM on 2-CTA pairs (M = 256 tcgen05 MMA)
   int r_splits, r_chunks_per_split;           // router: split of d into 32-wide chunks
   int g1_kb, g1_m_tiles;                      // gate/up GEMM: K blocks (d/128), 64-row tiles
   int g1_splits, g1_kb_per_split;             // gate/up K split (decode); 1 = SwiGLU epilogue

@@ -29,15 +29,15 @@ int num_sms() {
   return n;
 }
 
-// Smallest split count s (each split >= 4 K blocks) whose tile count fills the SMs' waves to
-// >= 90%; otherwise the best filling one.
-static int choose_splits(int64_t base_tiles, int num_kb) {
+// Smallest split count s (each split >= 4 K blocks) whose tile count fills the waves of `units`
+// persistent workers (SMs, or SM pairs) to >= 90%; otherwise the best filling one.
+static int choose_splits(int64_t base_tiles, int num_kb, int units = kPlanSMs) {
   const int max_s = std::max(1, std::min(32, num_kb / 4));
   int best = 1;
   double best_eff = 0.0;
   for (int s = 1; s <= max_s; ++s) {
     const int64_t tiles = base_tiles * s;
-    const double eff = double(tiles) / double(ceil_div(tiles, kPlanSMs) * kPlanSMs);
+    const double eff = double(tiles) / double(ceil_div(tiles, units) * units);
     if (eff >= 0.9) return s;
     if (eff > best_eff + 1e-9) {
       best_eff = eff;
@@ -74,6 +74,16 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
   BN = MOE_FORCE_BN;
 #endif
   p->BN = BN;
+  // Prefill-sized token tiles run on SM pairs: the pair's M = 256 MMA shares one token tile
+  // between two SMs (each loads half of it), so a token row crosses L2 -> shared memory once per
+  // 256 weight rows instead of once per 128. That pays when the tiles are full (BN >= 192, i.e.
+  // >= ~100 rows per active expert) and, for the down GEMM, when K = F is long enough (>= 16 K
+  // blocks) for the main loop rather than the epilogue to set the pace.
+  p->pair1 = BN >= 192;
+  p->pair2 = BN >= 192 && ceil_div(F, kBK) >= 16;
+#ifdef MOE_FORCE_PAIR
+  p->pair1 = p->pair2 = MOE_FORCE_PAIR;
+#endif
 
   // router: 32x32 tiles; split d so that the grid covers about two waves
   const int64_t rtiles = ceil_div(std::max(T, 1), kRouterTile) * ceil_div(E, kRouterTile);
@@ -98,7 +108,8 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
     p->g1_kb_per_split = (int)ceil_div(p->g1_kb, s1);
     p->g1_splits = (int)ceil_div(p->g1_kb, p->g1_kb_per_split);
   }
-  int s2 = choose_splits(est_ntiles * p->g2_m_tiles, p->g2_kb);
+  int s2 = p->pair2 ? choose_splits(est_ntiles * ceil_div(p->g2_m_tiles, 2), p->g2_kb, kPlanSMs / 2)
+                   : choose_splits(est_ntiles * p->g2_m_tiles, p->g2_kb);
   p->g2_kb_per_split = (int)ceil_div(p->g2_kb, s2);
   p->g2_splits = (int)ceil_div(p->g2_kb, p->g2_kb_per_split);   // every split non-empty
 

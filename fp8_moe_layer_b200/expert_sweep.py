@@ -58,6 +58,7 @@ def main():
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             flush_rd.sum()
+            torch.cuda._sleep(400_000)     # ~0.2 ms: the host enqueues the step meanwhile
             ev[i][0].record()
             layer(h)
             ev[i][1].record()

@@ -22,8 +22,10 @@ class MoEGraphExecutor:
     """Replays captured moe_forward graphs for a device-resident layer (ops.MoELayerFP8)."""
 
     def __init__(self, layer: "ops.MoELayerFP8", buckets: Sequence[int] = (1, 2, 4, 8, 16, 32, 64,
-                                                                          128, 256, 512)):
+                                                                          128, 256, 512),
+                 k: Optional[int] = None):
         self.layer = layer
+        self.k = layer.shape.k if k is None else int(k)   # the fixed-k profile's k
         self.buckets = sorted(set(int(b) for b in buckets))
         self.graphs: Dict[Tuple[int, str], dict] = {}
         self.stream = torch.cuda.Stream(device=layer.device)
@@ -45,7 +47,7 @@ class MoEGraphExecutor:
         ops.clear_status(ws)
 
         def run():
-            ops.moe_forward(h, layer.router_w, layer.router_bias, s.k, kpt, layer.w13,
+            ops.moe_forward(h, layer.router_w, layer.router_bias, self.k, kpt, layer.w13,
                             layer.w13_scale, layer.w2, layer.w2_scale, s.k_max,
                             shared=layer.shared, ws=ws, y=y)
 
@@ -62,7 +64,7 @@ class MoEGraphExecutor:
     def __call__(self, hidden: torch.Tensor, k_per_token: Optional[torch.Tensor] = None):
         T = hidden.shape[0]
         elastic = k_per_token is not None
-        key = (self.bucket(T), "elastic" if elastic else f"k{self.layer.shape.k}")
+        key = (self.bucket(T), "elastic" if elastic else f"k{self.k}")
         if key not in self.graphs:
             self.graphs[key] = self._capture(key[0], elastic)
         g = self.graphs[key]

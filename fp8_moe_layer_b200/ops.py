@@ -279,10 +279,14 @@ class MoELayerFP8:
         self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
         clear_status(self.ws)
 
-    def __call__(self, hidden, k_per_token=None, y=None, debug=False, stage_events=None):
+    def __call__(self, hidden, k_per_token=None, y=None, debug=False, stage_events=None,
+                 k: Optional[int] = None):
+        """y = layer(hidden); per-token k from ``k_per_token`` if given, else the fixed ``k``
+        (default: the layer's k)."""
         if hidden.shape[0] > self.max_T:
             raise ValueError("more tokens than the workspace was sized for")
-        return moe_forward(hidden, self.router_w, self.router_bias, self.shape.k, k_per_token,
+        k = self.shape.k if k is None else int(k)
+        return moe_forward(hidden, self.router_w, self.router_bias, k, k_per_token,
                            self.w13, self.w13_scale, self.w2, self.w2_scale, self.shape.k_max,
                            shared=self.shared, ws=self.ws, y=y, debug=debug,
                            stage_events=stage_events)

@@ -61,6 +61,12 @@ SMALL = [
     I.MoEShape("single_expert", 45, 128, 1, 128, 1, 1),
     I.MoEShape("ragged_K_F", 29, 192, 5, 96, 2, 2),
     I.MoEShape("small_d", 12, 64, 4, 32, 2, 2),
+    # token tiles >= 192 rows run the gate/up GEMM on 2-SM pairs, and the down GEMM too when
+    # F >= 2048: odd weight m-tile counts (F = 192 -> 3 gate/up tiles, d = 384 -> 3 down tiles;
+    # the pair's second half falls off the matrix), ragged tails, a shared-expert group
+    I.MoEShape("pair_odd_m", 260, 384, 4, 192, 2, 2, zipf_s=0.5),
+    I.MoEShape("pair_shared", 280, 256, 4, 128, 2, 2, F_shared=128),
+    I.MoEShape("pair_down_odd_m", 160, 384, 2, 2048, 2, 2),
 ]
 
 
