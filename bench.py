@@ -141,6 +141,15 @@ def algorithmic(shape, offsets: np.ndarray):
     return dict(active_experts=active, routed_rows=R, bytes=B, flops=flops, gemm1_bytes=g1_bytes)
 
 
+def kernel_src_digest() -> str:
+    """sha256 (first 16 hex digits) over the sources the grouped GEMM kernels are compiled from."""
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "common.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "fp8_moe_layer_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def ncu_traffic(kernel_tag: str):
     """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged
     since it was captured (else None)."""
@@ -149,9 +158,7 @@ def ncu_traffic(kernel_tag: str):
         return None
     with open(path) as f:
         rec = json.load(f)
-    src = os.path.join(ROOT, "fp8_moe_layer_b200", "csrc", "gemm.cu")
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if rec.get("gemm_cu_sha256_16") != digest:
+    if rec.get("kernel_src_sha256_16") != kernel_src_digest():
         return None
     return rec.get("dram_bytes_per_launch")
 

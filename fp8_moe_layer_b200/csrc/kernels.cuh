@@ -57,7 +57,8 @@ struct GemmArgs {
   int* status;
 };
 
-int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p);
+// k_est: experts per token the GEMM tiles are planned for (0 = k_max); buffers are for k_max.
+int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est = 0);
 
 cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
                                  float* part, cudaStream_t s);

@@ -29,25 +29,29 @@ int num_sms() {
   return n;
 }
 
-// Smallest split count s (each split >= 4 K blocks) whose tile count fills the waves of `units`
-// persistent workers (SMs, or SM pairs) to >= 90%; otherwise the best filling one.
-static int choose_splits(int64_t base_tiles, int num_kb, int units = kPlanSMs) {
+// K-split count of a grouped GEMM: the s (each split >= 4 K blocks) that minimises the estimated
+// HBM time -- ceil(tiles * s / units) waves of tiles that each read w_tile / s weight bytes and
+// write out_tile output bytes (plus a fixed per-tile cost), and the read-back of the s partial
+// sums by the kernel that reduces them.
+static int choose_splits(int64_t base_tiles, int num_kb, int units, double w_tile,
+                         double out_tile) {
+  constexpr double kTileOverheadBytes = 32e3;
   const int max_s = std::max(1, std::min(32, num_kb / 4));
   int best = 1;
-  double best_eff = 0.0;
+  double best_cost = 0.0;
   for (int s = 1; s <= max_s; ++s) {
-    const int64_t tiles = base_tiles * s;
-    const double eff = double(tiles) / double(ceil_div(tiles, units) * units);
-    if (eff >= 0.9) return s;
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
+    const double waves = (double)ceil_div(base_tiles * s, units);
+    const double cost = waves * (w_tile / s + out_tile + kTileOverheadBytes) +
+                        (double)base_tiles * s * out_tile / units;
+    if (s == 1 || cost < best_cost * (1.0 - 1e-9)) {
+      best_cost = cost;
       best = s;
     }
   }
   return best;
 }
 
-int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
+int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est) {
   if (T < 0 || d < 16 || d % 16 || F < 16 || F % 16 || E < 1 || k_max < 1) return MOE_ERR_INVALID_ARG;
   if (E > kMaxExperts || k_max > kMaxK) return MOE_ERR_UNSUPPORTED;
   if (Fs < 0) return MOE_ERR_INVALID_ARG;
@@ -63,9 +67,12 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
 
   // token tile: the smallest of {16, 32, 64, 128, 192, 256} >= 1.25 x the mean rows of an active
   // expert. A tile only loads and multiplies its valid rows, so a tile larger than the group
-  // costs shared memory (fewer pipeline stages), not traffic.
-  const int64_t active = std::max<int64_t>(1, std::min<int64_t>(E, routed));
-  const double mean_rows = double(routed) / double(active);
+  // costs shared memory (fewer pipeline stages), not traffic. The tiles are planned for k_est
+  // experts per token (the fixed k, or an estimate of the mean k_t of an elastic batch); the
+  // buffers for k_max.
+  const int64_t routed_est = (int64_t)T * std::max(1, std::min(k_est > 0 ? k_est : k_max, k_max));
+  const int64_t active = std::max<int64_t>(1, std::min<int64_t>(E, routed_est));
+  const double mean_rows = double(routed_est) / double(active);
   static const int kTiles[] = {16, 32, 64, 128, 192, 256};
   int BN = 256;
   for (int t : kTiles)
@@ -101,15 +108,19 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p) {
   p->g1_kb_per_split = p->g1_kb;
   p->g2_kb = (int)ceil_div(F, kBK);
   p->g2_m_tiles = (int)ceil_div(d, 128);
-  const int64_t est_ntiles = std::max<int64_t>(active, ceil_div(routed, BN)) +
+  const int64_t est_ntiles = std::max<int64_t>(active, ceil_div(routed_est, BN)) +
                              (p->shared ? ceil_div(T, BN) : 0);
-  if (BN <= 64) {
-    const int s1 = choose_splits(est_ntiles * p->g1_m_tiles, p->g1_kb);
+  const double tile_rows = std::min<double>(BN, mean_rows);
+  if (BN <= 64) {   // gate/up partials: 64 gate + 64 up fp32 columns per routed row
+    const int s1 = choose_splits(est_ntiles * p->g1_m_tiles, p->g1_kb, kPlanSMs, 128.0 * d,
+                                 tile_rows * 128 * 4);
     p->g1_kb_per_split = (int)ceil_div(p->g1_kb, s1);
     p->g1_splits = (int)ceil_div(p->g1_kb, p->g1_kb_per_split);
   }
-  int s2 = p->pair2 ? choose_splits(est_ntiles * ceil_div(p->g2_m_tiles, 2), p->g2_kb, kPlanSMs / 2)
-                   : choose_splits(est_ntiles * p->g2_m_tiles, p->g2_kb);
+  const int m_rows2 = p->pair2 ? 256 : 128;      // weight rows of one down-GEMM work unit
+  int s2 = choose_splits(est_ntiles * ceil_div(p->g2_m_tiles, m_rows2 / 128), p->g2_kb,
+                         p->pair2 ? kPlanSMs / 2 : kPlanSMs, (double)m_rows2 * F,
+                         tile_rows * m_rows2 * 4);
   p->g2_kb_per_split = (int)ceil_div(p->g2_kb, s2);
   p->g2_splits = (int)ceil_div(p->g2_kb, p->g2_kb_per_split);   // every split non-empty
 
@@ -392,10 +403,16 @@ extern "C" {
 
 size_t moe_workspace_bytes(const moe_dims* dims) {
   if (!dims) return 0;
-  Plan p;
-  if (plan_make(dims->T, dims->d, dims->E, dims->F, dims->k_max, dims->F_shared, &p) != MOE_OK)
-    return 0;
-  return p.bytes;
+  // the largest need over the tile plans moe_forward may use (fixed k = 1 .. k_max, or the
+  // elastic estimate k_max / 2)
+  size_t need = 0;
+  for (int k = 1; k <= std::max(1, dims->k_max); ++k) {
+    Plan p;
+    if (plan_make(dims->T, dims->d, dims->E, dims->F, dims->k_max, dims->F_shared, &p, k) != MOE_OK)
+      return 0;
+    need = std::max(need, p.bytes);
+  }
+  return need;
 }
 
 const char* moe_status_string(int status) {
@@ -540,7 +557,9 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                 size_t ws_bytes, void* stream, const moe_debug_out* dbg) {
   if (!dims) return MOE_ERR_INVALID_ARG;
   Plan p;
-  MOE_TRY(plan_make(dims->T, dims->d, dims->E, dims->F, dims->k_max, dims->F_shared, &p));
+  // tiles planned for the fixed k, or for k_max / 2 experts per token of an elastic batch
+  const int k_est = k_per_token ? std::max(1, dims->k_max / 2) : k;
+  MOE_TRY(plan_make(dims->T, dims->d, dims->E, dims->F, dims->k_max, dims->F_shared, &p, k_est));
   if (p.T == 0) return MOE_OK;
   if (!hidden || !router_w || !w13 || !w13_scale || !w2 || !w2_scale || !y) return MOE_ERR_INVALID_ARG;
   if (p.shared && (!w13_shared || !w13s_scale || !w2_shared || !w2s_scale)) return MOE_ERR_INVALID_ARG;

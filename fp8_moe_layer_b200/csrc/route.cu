@@ -91,8 +91,16 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
 
   if (do_route) {
     for (int e = tid; e < E; e += 128) {
-      float v = 0.f;
-      for (int s = 0; s < splits; ++s) v += part[((size_t)s * T + t) * E + e];
+      // split partials in fixed order: eight independent accumulators keep eight loads in
+      // flight (a decode batch splits d finely, and these loads are the kernel's latency)
+      float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      int s = 0;
+      for (; s + 8 <= splits; s += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a8[u] += part[((size_t)(s + u) * T + t) * E + e];
+      }
+      for (int u = 0; s < splits; ++s, ++u) a8[u] += part[((size_t)s * T + t) * E + e];
+      float v = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
       if (bias) v += bias[e];
       lg[e] = v;
     }
@@ -103,9 +111,10 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
       if (tid == 0) report(status, kStatusDeviceCheck, kWhereRoute, t);
       kt = max(1, min(kt, kcap));
     }
+    __shared__ int cand[kMaxCandidates];
+    __shared__ int ncand;
+    bool by_cand = false;          // exact selection over the refined candidates only
     if (refine_w) {
-      __shared__ int cand[kMaxCandidates];
-      __shared__ int ncand;
       __shared__ float vk_s;
       if (warp == 0) {
         // approximate k_t-th largest logit
@@ -156,6 +165,7 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
         const int e = all ? c : cand[c];
         const float4* wr = reinterpret_cast<const float4*>(refine_w + (size_t)e * d);
         float acc = 0.f;
+#pragma unroll 8
         for (int i = lane; i < nv; i += 32) {
           const uint4 v = xr[i];
           const float4 a = __ldg(wr + 2 * i), b = __ldg(wr + 2 * i + 1);
@@ -174,15 +184,20 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
         if (lane == 0) lg[e] = acc + (bias ? bias[e] : 0.f);
       }
       __syncthreads();
+      by_cand = !all;
     }
     if (warp == 0) {
-      uint32_t taken = 0;            // bit i: expert lane + 32*i already selected
+      // bit i of `taken`: scan slot lane + 32 i already selected (slot = expert, or candidate
+      // index when the refined candidates are scanned; the others hold -inf then)
+      uint32_t taken = 0;
       float sel_v = 0.f;             // lane j keeps the j-th selected logit
       int sel_e = -1;
+      const int n_scan = by_cand ? ncand : E;
       for (int j = 0; j < kt; ++j) {
         float bv = -INFINITY;
         int be = 0x7FFFFFFF;
-        for (int i = 0, e = lane; e < E; ++i, e += 32) {
+        for (int i = 0, c = lane; c < n_scan; ++i, c += 32) {
+          const int e = by_cand ? cand[c] : c;
           const float v = lg[e];
           if (!((taken >> i) & 1u) && (v > bv || (v == bv && e < be))) {
             bv = v;
@@ -198,7 +213,12 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
             be = oe;
           }
         }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        if (by_cand) {
+          for (int i = 0, c = lane; c < n_scan; ++i, c += 32)
+            if (cand[c] == be) taken |= 1u << i;
+        } else if ((be & 31) == lane) {
+          taken |= 1u << (be >> 5);
+        }
         if (lane == j) {
           sel_v = bv;
           sel_e = be;
