@@ -71,9 +71,15 @@ cudaError_t launch_topk_quant(const Plan& p, const float* part, const float* bia
 // logits + topk_quant.
 // (the fused router holds a token's row in registers: d <= 8192)
 inline bool router_is_fused(int E, int d) { return E <= 32 && d <= 8192; }
-inline bool router_uses_mma(int E, int T) { return E > 32 && T >= 64; }
+// Router logits on the tensor cores (three bf16 planes + exact refinement of the candidates) once
+// the fp32 CUDA-core work 2·T·E·d is large: measured on B200, the exact CUDA-core router is faster
+// up to T·E·d ~ 2.4e8 (Qwen3 T=64, DeepSeek T=128, MoE-Prism T=64) and the tensor-core one from
+// ~1.1e9 (Qwen3 T=4096, MoE-Prism T=2048, DeepSeek T=8192); the switch sits at 2^29.
+inline bool router_uses_mma(int E, int T, int d) {
+  return E > 32 && (long long)T * E * d >= (1LL << 29);
+}
 inline bool router_is_fused(const Plan& p) { return router_is_fused(p.E, p.d); }
-inline bool router_uses_mma(const Plan& p) { return router_uses_mma(p.E, p.T); }
+inline bool router_uses_mma(const Plan& p) { return router_uses_mma(p.E, p.T, p.d); }
 // planes: 3 * E * d bf16 (workspace); map_w over planes [3][E][d], map_x over hidden [T][d]
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
                               const CUtensorMap& map_w, const CUtensorMap& map_x, float* logits,
@@ -84,6 +90,13 @@ cudaError_t launch_route_fused(const Plan& p, const uint16_t* hidden, const floa
                                int* status, cudaStream_t s);
 // scratch: 2 * permute_blocks(p) * E int32 (per-block counts and bases; unused for one block)
 int permute_blocks(const Plan& p);
+// grouping + row gather in one kernel (when the grouping fits one block, T * k_max <= 8192)
+bool permute_gather_fused(const Plan& p);
+cudaError_t launch_permute_gather(const Plan& p, const int32_t* ids, int k,
+                                  const int32_t* k_per_token, int32_t* offsets, int32_t* perm,
+                                  int32_t* inv, int32_t* tiles, const uint8_t* xq, const float* xs,
+                                  uint8_t* xqp, float* xsp, uint32_t* amax, int* status,
+                                  cudaStream_t s);
 cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
                            int32_t* scratch, int* status, cudaStream_t s);

@@ -96,7 +96,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   const int64_t rtiles = ceil_div(std::max(T, 1), kRouterTile) * ceil_div(E, kRouterTile);
   const int nchunks = (int)ceil_div(d, kRouterTile);
   int rs = (int)std::min<int64_t>(nchunks, std::max<int64_t>(1, ceil_div(2 * kPlanSMs, rtiles)));
-  if (router_uses_mma(E, T)) rs = 1;      // the tensor-core router writes whole logits
+  if (router_uses_mma(E, T, d)) rs = 1;      // the tensor-core router writes whole logits
   p->r_chunks_per_split = (int)ceil_div(nchunks, rs);
   p->r_splits = (int)ceil_div(nchunks, p->r_chunks_per_split);
 
@@ -144,7 +144,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   p->off_aq = take((size_t)p->Rpad * F);
   p->off_s2 = take(sizeof(float) * (size_t)p->Rpad);
   p->off_o = take(sizeof(float) * (size_t)p->g2_splits * p->Rpad * d);
-  p->off_planes = take(router_uses_mma(E, T) ? 3 * sizeof(uint16_t) * (size_t)E * d : 0);
+  p->off_planes = take(router_uses_mma(E, T, d) ? 3 * sizeof(uint16_t) * (size_t)E * d : 0);
   p->off_hpart = take(p->g1_splits > 1 ? sizeof(float) * p->g1_splits * (size_t)p->Rcap * 2 * F : 0);
   p->bytes = off;
   return MOE_OK;
@@ -317,7 +317,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
                    const uint8_t* w2, const float* w2_scale, const uint8_t* w13s,
                    const float* w13s_scale, const uint8_t* w2s, const float* w2s_scale,
                    float* o, size_t split_stride, int64_t o_rows, void* const* ev,
-                   cudaStream_t s) {
+                   cudaStream_t s, bool gathered = false) {
   CUtensorMap m13, m13s, mxq64, mxq16, m2, m2s, maq64, maq16;
   if (!map_w13(&m13, w13, p.E, p.F, p.d) || !map_w2(&m2, w2, p.E, p.d, p.F) ||
       !map_rows(&mxq64, w.xqp, p.Rpad, p.d, 64) || !map_rows(&mxq16, w.xqp, p.Rpad, p.d, 16) ||
@@ -336,7 +336,8 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   const int32_t* total_rows = w.offsets + p.G;     // offsets[G] = routed (+ shared) rows
 
   record(3);
-  MOE_CUDA(launch_gather(p, w.xq, w.xs, w.perm, total_rows, w.xqp, w.xsp, w.amax, w.status, s));
+  if (!gathered)   // (else the grouping kernel already laid the rows out)
+    MOE_CUDA(launch_gather(p, w.xq, w.xs, w.perm, total_rows, w.xqp, w.xsp, w.amax, w.status, s));
 
   GemmArgs g1{};
   g1.group_offsets = w.offsets;
@@ -592,11 +593,16 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                                w.status, s));
   }
   record(2);
-  MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
-                          w.status, s));
+  const bool fused = permute_gather_fused(p);
+  if (fused)
+    MOE_CUDA(launch_permute_gather(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles,
+                                   w.xq, w.xs, w.xqp, w.xsp, w.amax, w.status, s));
+  else
+    MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
+                            w.status, s));
   const size_t split_stride = (size_t)p.Rpad * p.d;
   MOE_TRY(run_ffn(p, w, w13, w13_scale, w2, w2_scale, w13_shared, w13s_scale, w2_shared,
-                  w2s_scale, w.o, split_stride, p.Rcap, ev, s));
+                  w2s_scale, w.o, split_stride, p.Rcap, ev, s, fused));
   record(7);
   MOE_CUDA(launch_combine(p, w.o, p.g2_splits, split_stride, w.w, w.inv,
                           p.shared ? w.o : nullptr, p.shared ? w.offsets + p.E : nullptr,

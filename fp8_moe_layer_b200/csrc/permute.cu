@@ -43,18 +43,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& 
   return r;
 }
 
-// Single block. Warp w owns tokens [w*chunk, (w+1)*chunk) and walks its (token, slot) pairs in
-// token-major order, 32 at a time. Lanes holding the same expert find each other with
-// __match_any_sync; a lane's rank among them plus the warp's running cursor for that expert
-// gives its row, so rows inside an expert are in ascending token order.
-__global__ void __launch_bounds__(kPermThreads) permute_kernel(
-    const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
-    int E, int has_shared, int BN, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
-    int32_t* __restrict__ inv, int32_t* __restrict__ tiles, int* status) {
-  pdl_wait();      // predecessor kernel complete, its writes visible
-  pdl_trigger();   // let the next kernel launch
-  extern __shared__ int hist[];                  // [kPermWarps][E]
-  __shared__ int warp_sums[33];
+// One block computes the whole grouping. Warp w owns tokens [w*chunk, (w+1)*chunk) and walks its
+// (token, slot) pairs in token-major order, 32 at a time. Lanes holding the same expert find each
+// other with __match_any_sync; a lane's rank among them plus the warp's running cursor for that
+// expert gives its row, so rows inside an expert are in ascending token order. `write` selects
+// the block that stores offsets / perm / inv / tiles (and reports bad ids); `s_perm`, when given,
+// receives perm[] in shared memory. Returns the routed row count R.
+__device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_max, int k,
+                                  const int32_t* __restrict__ k_per_token, int E, int has_shared,
+                                  int BN, int32_t* __restrict__ offsets,
+                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                  int32_t* __restrict__ tiles, int* status, int* hist,
+                                  int* warp_sums, int* s_perm, bool write) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kPermWarps * E; i += kPermThreads) hist[i] = 0;
   __syncthreads();
@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
       if (j < kt) {
         const int e = ids[idx];
         if (e >= 0 && e < E) atomicAdd(&my_hist[e], 1);
-        else report(status, kStatusDeviceCheck, kWherePermute, t);
+        else if (write) report(status, kStatusDeviceCheck, kWherePermute, t);
       }
     }
   }
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
       for (int w = 0; w < kPermWarps; ++w) cnt += hist[w * E + e];
     const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
     if (e < E) {
-      offsets[e] = off;
+      if (write) offsets[e] = off;
       int run = off;
       for (int w = 0; w < kPermWarps; ++w) {
         const int c = hist[w * E + e];
@@ -98,8 +98,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     }
     const int nt = e < E ? (cnt + BN - 1) / BN : 0;
     const int toff = block_exclusive_scan(nt, warp_sums, total_tiles);
-    if (e < E) tiles[e] = toff;
-    if (threadIdx.x == 0) {
+    if (write && e < E) tiles[e] = toff;
+    if (write && threadIdx.x == 0) {
       offsets[E] = total_rows;
       if (has_shared) {
         offsets[E + 1] = total_rows + T;
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
         e = ids[idx];
         valid = e >= 0 && e < E;
       }
-      if (!valid) inv[idx] = -1;
+      if (!valid && write) inv[idx] = -1;
     }
     const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : E + lane);
     const int rank = __popc(peers & ((1u << lane) - 1u));
@@ -133,14 +133,68 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     __syncwarp();
     if (valid) {
       const int r = cursor + rank;
-      perm[r] = t;
-      inv[idx] = r;
+      if (write) {
+        perm[r] = t;
+        inv[idx] = r;
+      }
+      if (s_perm) s_perm[r] = t;
       if (rank == 0) my_hist[e] = cursor + __popc(peers);
     }
     __syncwarp();
   }
   if (has_shared)
-    for (int t = threadIdx.x; t < T; t += kPermThreads) perm[total_rows + t] = t;
+    for (int t = threadIdx.x; t < T; t += kPermThreads) {
+      if (write) perm[total_rows + t] = t;
+      if (s_perm) s_perm[total_rows + t] = t;
+    }
+  return total_rows;
+}
+
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(
+    const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
+    int E, int has_shared, int BN, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv, int32_t* __restrict__ tiles, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  extern __shared__ int hist[];                  // [kPermWarps][E]
+  __shared__ int warp_sums[33];
+  permute_block_body(ids, T, k_max, k, k_per_token, E, has_shared, BN, offsets, perm, inv, tiles,
+                     status, hist, warp_sums, nullptr, true);
+}
+
+// Grouping and row gather in one kernel, for batches whose grouping fits one block (T * k_max <=
+// 8192): every block computes the (small) grouping itself into shared memory -- so no block
+// waits for another -- block 0 also stores it, and each block then copies its share of the
+// quantised token rows into grouped order (one warp per row): xqp[r, :] = xq[perm[r], :],
+// xsp[r] = xs[perm[r]], amax[r] = 0. Saves the separate gather launch and its dependency wait.
+__global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(
+    const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
+    int E, int has_shared, int BN, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv, int32_t* __restrict__ tiles, const uint8_t* __restrict__ xq,
+    const float* __restrict__ xs, int d, uint8_t* __restrict__ xqp, float* __restrict__ xsp,
+    uint32_t* __restrict__ amax, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  extern __shared__ int smem_i[];                // hist [kPermWarps][E], then perm [rows]
+  __shared__ int warp_sums[33];
+  int* hist = smem_i;
+  int* s_perm = smem_i + kPermWarps * E;
+  const int R = permute_block_body(ids, T, k_max, k, k_per_token, E, has_shared, BN, offsets, perm,
+                                   inv, tiles, status, hist, warp_sums, s_perm, blockIdx.x == 0);
+  __syncthreads();
+  const int rows = R + (has_shared ? T : 0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nv = d / 16;
+  for (int r = blockIdx.x * kPermWarps + warp; r < rows; r += gridDim.x * kPermWarps) {
+    const int t = s_perm[r];
+    const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xqp + (size_t)r * d);
+    for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+    if (lane == 0) {
+      xsp[r] = xs[t];
+      amax[r] = 0u;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -390,6 +444,34 @@ cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32
   launch_pdl(permute_scatter_kernel, dim3(blocks), dim3(kPermBlkThreads), smem, s, ids, p.T, p.k_max, k, k_per_token,
                                                                p.E, p.shared ? 1 : 0, bbase,
                                                                offsets, perm, inv);
+  return cudaGetLastError();
+}
+
+bool permute_gather_fused(const Plan& p) { return permute_blocks(p) == 1; }
+
+cudaError_t launch_permute_gather(const Plan& p, const int32_t* ids, int k,
+                                  const int32_t* k_per_token, int32_t* offsets, int32_t* perm,
+                                  int32_t* inv, int32_t* tiles, const uint8_t* xq, const float* xs,
+                                  uint8_t* xqp, float* xsp, uint32_t* amax, int* status,
+                                  cudaStream_t s) {
+  // T * k_max <= 8192 here, so rows = T * k_max (+ T) <= 16384
+  const size_t smem = sizeof(int) * ((size_t)kPermWarps * p.E + (size_t)p.Rcap);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(permute_gather_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(int) * (kPermWarps * kMaxExperts + 16384));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  // about 32 KB of rows per block (one warp per row), at most one block per SM
+  const int64_t bytes = p.Rcap * (int64_t)p.d;
+  const int grid = (int)std::min<int64_t>(std::max<int64_t>((bytes + 32767) / 32768, 1), num_sms());
+  launch_pdl(permute_gather_kernel, dim3(grid), dim3(kPermThreads), smem, s, ids, p.T, p.k_max, k,
+             k_per_token, p.E, p.shared ? 1 : 0, p.BN, offsets, perm, inv, tiles, xq, xs, p.d,
+             xqp, xsp, amax, status);
   return cudaGetLastError();
 }
 

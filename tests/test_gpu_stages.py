@@ -12,9 +12,10 @@ pytestmark = pytest.mark.gpu
 
 ROUTE_SHAPES = [
     I.WORKLOADS["tiny_T16"],
-    I.MoEShape("cuda_core_router", 37, 256, 64, 64, 6, 6, zipf_s=0.8),     # E > 32, T < 64
-    I.MoEShape("mma_router_ragged_E", 100, 320, 48, 64, 4, 4),              # E % 128 != 0
-    I.MoEShape("mma_router_E33", 65, 128, 33, 64, 3, 3),
+    I.MoEShape("cuda_core_router", 37, 256, 64, 64, 6, 6, zipf_s=0.8),     # E > 32, small T·E·d
+    # the tensor-core router (T·E·d >= 2^29): E % 128 != 0 and T % 64 != 0, and E = 33
+    I.MoEShape("mma_router_ragged_E", 1000, 1056, 520, 64, 4, 4),
+    I.MoEShape("mma_router_E33", 8200, 2048, 33, 64, 3, 3),
     I.MoEShape("ragged", 37, 256, 6, 64, 2, 2),
     I.MoEShape("k_equals_E", 19, 128, 5, 64, 5, 5),
     I.WORKLOADS["qwen3_T64"],
