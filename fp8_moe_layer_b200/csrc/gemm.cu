@@ -103,7 +103,8 @@ __global__ void __launch_bounds__(256, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                         const __grid_constant__ CUtensorMap map_a_shared,
                         const __grid_constant__ CUtensorMap map_b64,
-                        const __grid_constant__ CUtensorMap map_b16, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap map_b16,
+                        const __grid_constant__ CUtensorMap map_out, const GemmArgs args) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   using C = GemmCfg<BN, MODE, PAIR>;
@@ -435,6 +436,7 @@ __global__ void __launch_bounds__(256, 1)
         // the accumulator wait); a shuffle hands column c's scale to the whole warp.
         constexpr int CW = C::CW;
         float* outp = args.out + (size_t)s * args.out_split_stride + (size_t)row0 * args.out_ld + ch;
+        const int split_rows = (int)(args.out_split_stride / (size_t)args.out_ld);   // map rows
 #pragma unroll 1
         for (int j = 0; !bad && j * CW < nvalid; ++j) {
           const int c0 = j * CW;
@@ -454,27 +456,37 @@ __global__ void __launch_bounds__(256, 1)
           for (int c = 0; c < CW; ++c)
             v[c] = __uint_as_float(r[c]) * __shfl_sync(0xffffffffu, rsv, c) * wsv;
           if constexpr (C::DOWN_T) {
-            // Through this warp's 32 x 33 block of shared memory: lane l then writes channels
-            // 4 (l % 8) .. +3 of token 4 i + l / 8 as one 16-byte store (a quarter of the store
-            // instructions of one 4-byte store per token; in this kernel the store instruction
-            // count, not the bytes, sets the pace of the epilogue).
-            float* tr = xchg + 32 * q * C::XCHG_LD;
-#pragma unroll
-            for (int c = 0; c < CW; ++c) tr[c * C::XCHG_LD + lane] = v[c];
+            // Through this warp's dense 32 x 32 fp32 block of shared memory (row = token): a full
+            // chunk leaves by one TMA tensor store, a ragged one by 16-byte stores of its valid
+            // rows. (In this kernel the count of global store instructions, not the bytes, set the
+            // epilogue's pace; the TMA store takes them off the SM's load/store path.)
+            float* tr = xchg + 32 * q * 32;
+            if (lane == 0) bulk_wait_read_all();       // the previous store has read the block
             __syncwarp();
-            const int chq = m * 128 + 32 * q, cc = 4 * (lane & 7);
-            float* base = args.out + (size_t)s * args.out_split_stride +
-                          (size_t)(row0 + c0) * args.out_ld + chq + cc;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int c = 4 * i + (lane >> 3);
-              if (c < ncol && chq + cc < args.M_valid) {
-                const float* t4 = tr + c * C::XCHG_LD + cc;
-                *reinterpret_cast<float4*>(base + (size_t)c * args.out_ld) =
-                    make_float4(t4[0], t4[1], t4[2], t4[3]);
+            for (int c = 0; c < CW; ++c) tr[c * 32 + lane] = v[c];
+            const int chq = m * 128 + 32 * q;
+            if (ncol == CW) {
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0 && chq < args.M_valid) {
+                tma_store_2d(&map_out, tr, chq, s * split_rows + row0 + c0);
+                bulk_commit();
               }
+            } else {
+              __syncwarp();
+              const int cc = 4 * (lane & 7);
+              float* base = args.out + (size_t)s * args.out_split_stride +
+                            (size_t)(row0 + c0) * args.out_ld + chq + cc;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int c = 4 * i + (lane >> 3);
+                if (c < ncol && chq + cc < args.M_valid)
+                  *reinterpret_cast<float4*>(base + (size_t)c * args.out_ld) =
+                      *reinterpret_cast<const float4*>(tr + c * 32 + cc);
+              }
+              __syncwarp();
             }
-            __syncwarp();
           } else if (valid) {
 #pragma unroll
             for (int c = 0; c < CW; ++c)
@@ -488,6 +500,9 @@ __global__ void __launch_bounds__(256, 1)
         if constexpr (PAIR) mbar_arrive_cluster(tempty_l + 8u * ab);   // the even CTA's barrier
         else mbar_arrive(&tempty[ab]);
       }
+    }
+    if constexpr (C::DOWN_T) {
+      if (lane == 0) bulk_wait_all();              // this warp's TMA stores have completed
     }
   }
 
@@ -504,7 +519,8 @@ __global__ void __launch_bounds__(256, 1)
 namespace {
 template <int BN, int MODE, bool PAIR>
 cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& ash, const CUtensorMap& b64,
-                          const CUtensorMap& b16, const GemmArgs& args, cudaStream_t s) {
+                          const CUtensorMap& b16, const CUtensorMap& out, const GemmArgs& args,
+                          cudaStream_t s) {
   using C = GemmCfg<BN, MODE, PAIR>;
   static int grid_cache[64] = {};
   int dev = 0;
@@ -538,33 +554,33 @@ cudaError_t launch_gemm_t(const CUtensorMap& a, const CUtensorMap& ash, const CU
     grid_cache[dev] = grid;
   }
   launch_pdl_cluster(grouped_gemm_kernel<BN, MODE, PAIR>, dim3(grid_cache[dev]), dim3(256), C::SMEM,
-                     PAIR ? 2 : 1, s, a, ash, b64, b16, args);
+                     PAIR ? 2 : 1, s, a, ash, b64, b16, out, args);
   return cudaGetLastError();
 }
 
 template <int MODE>
 cudaError_t launch_by_bn(int BN, bool pair, const CUtensorMap& a, const CUtensorMap& ash,
-                         const CUtensorMap& b64, const CUtensorMap& b16, const GemmArgs& args,
-                         cudaStream_t s) {
+                         const CUtensorMap& b64, const CUtensorMap& b16, const CUtensorMap& out,
+                         const GemmArgs& args, cudaStream_t s) {
   switch (BN) {
-    case 16: return launch_gemm_t<16, MODE, false>(a, ash, b64, b16, args, s);
-    case 32: return launch_gemm_t<32, MODE, false>(a, ash, b64, b16, args, s);
-    case 64: return launch_gemm_t<64, MODE, false>(a, ash, b64, b16, args, s);
+    case 16: return launch_gemm_t<16, MODE, false>(a, ash, b64, b16, out, args, s);
+    case 32: return launch_gemm_t<32, MODE, false>(a, ash, b64, b16, out, args, s);
+    case 64: return launch_gemm_t<64, MODE, false>(a, ash, b64, b16, out, args, s);
     default:
       if constexpr (MODE == kModeGateUpPartial) return cudaErrorInvalidValue;  // decode tiles only
       else {
         if (pair) {
           switch (BN) {
-            case 128: return launch_gemm_t<128, MODE, true>(a, ash, b64, b16, args, s);
-            case 192: return launch_gemm_t<192, MODE, true>(a, ash, b64, b16, args, s);
-            case 256: return launch_gemm_t<256, MODE, true>(a, ash, b64, b16, args, s);
+            case 128: return launch_gemm_t<128, MODE, true>(a, ash, b64, b16, out, args, s);
+            case 192: return launch_gemm_t<192, MODE, true>(a, ash, b64, b16, out, args, s);
+            case 256: return launch_gemm_t<256, MODE, true>(a, ash, b64, b16, out, args, s);
             default: return cudaErrorInvalidValue;
           }
         }
         switch (BN) {
-          case 128: return launch_gemm_t<128, MODE, false>(a, ash, b64, b16, args, s);
-          case 192: return launch_gemm_t<192, MODE, false>(a, ash, b64, b16, args, s);
-          case 256: return launch_gemm_t<256, MODE, false>(a, ash, b64, b16, args, s);
+          case 128: return launch_gemm_t<128, MODE, false>(a, ash, b64, b16, out, args, s);
+          case 192: return launch_gemm_t<192, MODE, false>(a, ash, b64, b16, out, args, s);
+          case 256: return launch_gemm_t<256, MODE, false>(a, ash, b64, b16, out, args, s);
           default: return cudaErrorInvalidValue;
         }
       }
@@ -575,14 +591,16 @@ cudaError_t launch_by_bn(int BN, bool pair, const CUtensorMap& a, const CUtensor
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
                                const CUtensorMap& acts64, const CUtensorMap& acts16,
                                const GemmArgs& a, bool partial, cudaStream_t s) {
-  if (partial) return launch_by_bn<kModeGateUpPartial>(p.BN, false, w13, w13s, acts64, acts16, a, s);
-  return launch_by_bn<kModeSwiGLU>(p.BN, p.pair1, w13, w13s, acts64, acts16, a, s);
+  // (the output map is used by the down GEMM only; the weight map stands in)
+  if (partial)
+    return launch_by_bn<kModeGateUpPartial>(p.BN, false, w13, w13s, acts64, acts16, w13, a, s);
+  return launch_by_bn<kModeSwiGLU>(p.BN, p.pair1, w13, w13s, acts64, acts16, w13, a, s);
 }
 
 cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
                              const CUtensorMap& acts64, const CUtensorMap& acts16,
-                             const GemmArgs& a, cudaStream_t s) {
-  return launch_by_bn<kModeDown>(p.BN, p.pair2, w2, w2s, acts64, acts16, a, s);
+                             const CUtensorMap& out, const GemmArgs& a, cudaStream_t s) {
+  return launch_by_bn<kModeDown>(p.BN, p.pair2, w2, w2s, acts64, acts16, out, a, s);
 }
 
 }  // namespace moe

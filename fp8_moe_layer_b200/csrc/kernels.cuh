@@ -115,7 +115,7 @@ cudaError_t launch_swiglu_requant(const Plan& p, const float* h, int splits, siz
                                   cudaStream_t s);
 cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtensorMap& w2s,
                              const CUtensorMap& acts64, const CUtensorMap& acts16,
-                             const GemmArgs& a, cudaStream_t s);
+                             const CUtensorMap& out, const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
                            const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s);
 cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t split_stride,

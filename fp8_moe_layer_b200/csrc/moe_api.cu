@@ -173,7 +173,8 @@ static EncodeTiledFn encode_fn() {
 // first; strides[i] is the byte stride of dimension i+1.
 static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                      const uint64_t* strides, const uint32_t* box,
-                     CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8) {
+                     CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -185,8 +186,18 @@ static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t*
     if (i + 1 < rank) gs[i] = strides[i];
   }
   return fn(m, dtype, rank, const_cast<void*>(base), gd, gs, bx, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// fp32 down-GEMM output [rows][d] (all K-split partials stacked): box 32 channels x 32 rows,
+// no swizzle, for the epilogue's TMA stores.
+static bool map_out(CUtensorMap* m, const float* o, int64_t rows, int d) {
+  const uint64_t dims[2] = {(uint64_t)d, (uint64_t)std::max<int64_t>(rows, 1)};
+  const uint64_t str[1] = {(uint64_t)d * 4};
+  const uint32_t box[2] = {32, 32};
+  return make_map(m, o, 2, dims, str, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // bf16 router weight planes [3][E][d]: box 64 (K) x 128 experts of one plane.
@@ -329,7 +340,6 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
     if (!map_w13(&m13s, w13s, 1, p.F, p.d) || !map_w2(&m2s, w2s, 1, p.d, p.F))
       return MOE_ERR_UNSUPPORTED;
   }
-  (void)o_rows;
   auto record = [&](int i) {
     if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
   };
@@ -391,8 +401,14 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g2.out_ld = p.d;
   g2.out_split_stride = split_stride;
   g2.row_amax = nullptr;
+  // the down GEMM's TMA stores: o as [splits x split rows][d] fp32 (a caller's unsplit buffer
+  // has exactly o_rows rows)
+  CUtensorMap mo;
+  const int64_t out_rows = p.g2_splits == 1 ? o_rows
+                                            : (int64_t)p.g2_splits * (int64_t)(split_stride / p.d);
+  if (!map_out(&mo, o, out_rows, p.d)) return MOE_ERR_UNSUPPORTED;
   record(6);
-  MOE_CUDA(launch_gemm_down(p, m2, m2s, maq64, maq16, g2, s));
+  MOE_CUDA(launch_gemm_down(p, m2, m2s, maq64, maq16, mo, g2, s));
   return MOE_OK;
 }
 
