@@ -80,6 +80,16 @@ inline bool router_uses_mma(int E, int T, int d) {
 }
 inline bool router_is_fused(const Plan& p) { return router_is_fused(p.E, p.d); }
 inline bool router_uses_mma(const Plan& p) { return router_uses_mma(p.E, p.T, p.d); }
+// decode batches (T <= 8) with E > 32: the one-kernel GEMV router (logits [T][E] in the
+// workspace's partial-logit buffer, the status word's counter for the last block)
+inline bool router_uses_gemv(int E, int T, int d) {
+  return E > 32 && T >= 1 && T <= 8 && !router_uses_mma(E, T, d);
+}
+inline bool router_uses_gemv(const Plan& p) { return router_uses_gemv(p.E, p.T, p.d); }
+cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
+                              const float* bias, int k, const int32_t* k_per_token, float* logits,
+                              int32_t* ids, float* w, uint8_t* xq, float* xs, bool do_quant,
+                              int* status, cudaStream_t s);
 // planes: 3 * E * d bf16 (workspace); map_w over planes [3][E][d], map_x over hidden [T][d]
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
                               const CUtensorMap& map_w, const CUtensorMap& map_x, float* logits,

@@ -480,6 +480,12 @@ int moe_route_topk(const moe_dims* dims, const uint16_t* hidden, const float* ro
                                 nullptr, nullptr, false, w.status, s));
     return MOE_OK;
   }
+  if (router_uses_gemv(p)) {
+    MOE_CUDA(cudaMemsetAsync(w.status + 3, 0, sizeof(int), s));   // the last-block counter
+    MOE_CUDA(launch_route_gemv(p, hidden, router_w, router_bias, k, k_per_token, w.part, topk_ids,
+                               topk_w, nullptr, nullptr, false, w.status, s));
+    return MOE_OK;
+  }
   MOE_TRY(run_router_logits(p, w, hidden, router_w, s));
   MOE_CUDA(launch_topk_quant(p, w.part, router_bias, k, k_per_token, topk_ids, topk_w, hidden,
                              nullptr, nullptr, true, false,
@@ -600,6 +606,11 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
     // one kernel for stages 0 and 1 (stage 1's events bracket nothing)
     MOE_CUDA(launch_route_fused(p, hidden, router_w, router_bias, k, k_per_token, w.ids, w.w, w.xq,
                                 w.xs, true, w.status, s));
+    record(1);
+  } else if (router_uses_gemv(p)) {
+    // decode batch: logits, top-k and quantisation in one kernel (stage 1's events bracket nothing)
+    MOE_CUDA(launch_route_gemv(p, hidden, router_w, router_bias, k, k_per_token, w.part, w.ids,
+                               w.w, w.xq, w.xs, true, w.status, s));
     record(1);
   } else {
     MOE_TRY(run_router_logits(p, w, hidden, router_w, s));

@@ -275,6 +275,164 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
   }
 }
 
+// Decode router (T <= 8 tokens, E > 32): one warp per expert computes that expert's logit for
+// every token (lane-strided chunks of 8 along d, fp32, then a butterfly; all loads in flight),
+// writes it to `logits` [T][E], and the last block to finish (a counter in the status word,
+// status[3]) selects the top-k, the weights and the FP8 quantisation of every token, then resets
+// the counter. One kernel instead of the tiled logits kernel (one global round trip per 32-wide
+// chunk of d) plus a separate top-k kernel.
+constexpr int kGemvMaxT = 8;
+
+template <int TT>
+__global__ void __launch_bounds__(256) route_gemv_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ W, const float* __restrict__ bias,
+    int T, int d, int E, int k, const int32_t* __restrict__ k_per_token, int k_max,
+    float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
+    uint8_t* __restrict__ xq, float* __restrict__ xs, int do_quant, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  __shared__ int s_last;
+  __shared__ float lg[kGemvMaxT][kMaxExperts];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int e = blockIdx.x * 8 + warp;
+  const int nv = d / 8;
+  if (e < E) {
+    float acc[TT];
+#pragma unroll
+    for (int j = 0; j < TT; ++j) acc[j] = 0.f;
+    const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
+#pragma unroll 4
+    for (int i = lane; i < nv; i += 32) {
+      const float4 a = __ldg(wr + 2 * i), b = __ldg(wr + 2 * i + 1);
+#pragma unroll
+      for (int j = 0; j < TT; ++j) {
+        if (j < T) {
+          const uint4 v = reinterpret_cast<const uint4*>(x + (size_t)j * d)[i];
+          float c8 = __uint_as_float(v.x << 16) * a.x;
+          c8 = fmaf(__uint_as_float(v.x & 0xFFFF0000u), a.y, c8);
+          c8 = fmaf(__uint_as_float(v.y << 16), a.z, c8);
+          c8 = fmaf(__uint_as_float(v.y & 0xFFFF0000u), a.w, c8);
+          c8 = fmaf(__uint_as_float(v.z << 16), b.x, c8);
+          c8 = fmaf(__uint_as_float(v.z & 0xFFFF0000u), b.y, c8);
+          c8 = fmaf(__uint_as_float(v.w << 16), b.z, c8);
+          c8 = fmaf(__uint_as_float(v.w & 0xFFFF0000u), b.w, c8);
+          acc[j] += c8;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < TT; ++j) {
+      if (j < T) {
+        float v = acc[j];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) logits[(size_t)j * E + e] = v + (bias ? bias[e] : 0.f);
+      }
+    }
+  }
+  // the last block to arrive sees every block's logits
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&status[3], 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (warp < T) {
+    const int t = warp;
+    float* my = lg[warp];
+    for (int ee = lane; ee < E; ee += 32) my[ee] = __ldcg(logits + (size_t)t * E + ee);
+    __syncwarp();
+    int kt = k_per_token ? k_per_token[t] : k;
+    const int kcap = min(E, k_max);
+    if (kt < 1 || kt > kcap) {
+      if (lane == 0) report(status, kStatusDeviceCheck, kWhereRoute, t);
+      kt = max(1, min(kt, kcap));
+    }
+    uint32_t taken = 0;            // bit i: expert lane + 32*i already selected
+    float sel_v = 0.f;             // lane j keeps the j-th selected logit
+    int sel_e = -1;
+    for (int j = 0; j < kt; ++j) {
+      float bv = -INFINITY;
+      int be = 0x7FFFFFFF;
+      for (int i = 0, ee = lane; ee < E; ++i, ee += 32) {
+        const float v = my[ee];
+        if (!((taken >> i) & 1u) && (v > bv || (v == bv && ee < be))) {
+          bv = v;
+          be = ee;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (lane == j) {
+        sel_v = bv;
+        sel_e = be;
+      }
+    }
+    const float lmax = __shfl_sync(0xffffffffu, sel_v, 0);
+    const float z = lane < kt ? expf(sel_v - lmax) : 0.f;
+    float zs = z;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
+    if (lane < k_max) {
+      ids[(size_t)t * k_max + lane] = lane < kt ? sel_e : -1;
+      wout[(size_t)t * k_max + lane] = lane < kt ? z / zs : 0.f;
+    }
+  }
+  if (do_quant) {
+    // the FP8 quantisation of each token by the whole block
+    __shared__ float red[8];
+    for (int t = 0; t < T; ++t) {
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+      float amax = 0.f;
+      for (int i = tid; i < nv; i += 256) {
+        const uint4 v = xr[i];
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] << 16)));
+          amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] & 0xFFFF0000u)));
+        }
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      if (lane == 0) red[warp] = amax;
+      __syncthreads();
+      float am = red[0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) am = fmaxf(am, red[w]);
+      __syncthreads();                                   // red[] is reused by the next token
+      const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
+      if (tid == 0) xs[t] = sc;
+      uint2* out = reinterpret_cast<uint2*>(xq + (size_t)t * d);
+      for (int i = tid; i < nv; i += 256) {
+        const uint4 v = xr[i];
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        uint32_t packed[2];
+#pragma unroll
+        for (int q = 0; q < 4; q += 2) {
+          const float a0 = __fdiv_rn(__uint_as_float(w4[q] << 16), sc);
+          const float a1 = __fdiv_rn(__uint_as_float(w4[q] & 0xFFFF0000u), sc);
+          const float a2 = __fdiv_rn(__uint_as_float(w4[q + 1] << 16), sc);
+          const float a3 = __fdiv_rn(__uint_as_float(w4[q + 1] & 0xFFFF0000u), sc);
+          packed[q / 2] = static_cast<uint32_t>(e4m3x2(a0, a1)) |
+                          (static_cast<uint32_t>(e4m3x2(a2, a3)) << 16);
+        }
+        out[i] = make_uint2(packed[0], packed[1]);
+      }
+    }
+  }
+  if (tid == 0) status[3] = 0;             // the counter is ready for the next launch
+}
+
 // Small-E router (E <= 32), one 256-thread block per token, fully fused: logits, top-k, weights
 // and the token's FP8 quantisation. Thread i accumulates x[t, 8c..8c+7] . W[e, 8c..8c+7] for the
 // chunks c = i, i + 256, ... (fp32), a butterfly inside each warp and a fixed-order sum over the
@@ -431,6 +589,27 @@ cudaError_t launch_route_fused(const Plan& p, const uint16_t* hidden, const floa
   else
     launch_pdl(route_block_kernel<32>, dim3(p.T), dim3(256), 0, s, hidden, router_w, bias, p.T,
                p.d, p.E, k, k_per_token, p.k_max, ids, w, xq, xs, q, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
+                              const float* bias, int k, const int32_t* k_per_token, float* logits,
+                              int32_t* ids, float* w, uint8_t* xq, float* xs, bool do_quant,
+                              int* status, cudaStream_t s) {
+  const dim3 grid((p.E + 7) / 8);
+  const int q = do_quant ? 1 : 0;
+  if (p.T <= 1)
+    launch_pdl(route_gemv_kernel<1>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
+               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
+  else if (p.T <= 2)
+    launch_pdl(route_gemv_kernel<2>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
+               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
+  else if (p.T <= 4)
+    launch_pdl(route_gemv_kernel<4>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
+               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
+  else
+    launch_pdl(route_gemv_kernel<8>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
+               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
   return cudaGetLastError();
 }
 

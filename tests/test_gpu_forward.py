@@ -61,6 +61,9 @@ SMALL = [
     I.MoEShape("single_expert", 45, 128, 1, 128, 1, 1),
     I.MoEShape("ragged_K_F", 29, 192, 5, 96, 2, 2),
     I.MoEShape("small_d", 12, 64, 4, 32, 2, 2),
+    # decode batches with E > 32 (the one-kernel GEMV router)
+    I.MoEShape("decode_gemv_T3", 3, 256, 96, 128, 6, 6, zipf_s=1.0),
+    I.MoEShape("decode_gemv_T8_shared", 8, 256, 40, 128, 4, 4, F_shared=128),
     # token tiles >= 192 rows run the gate/up GEMM on 2-SM pairs, and the down GEMM too when
     # F >= 2048: odd weight m-tile counts (F = 192 -> 3 gate/up tiles, d = 384 -> 3 down tiles;
     # the pair's second half falls off the matrix), ragged tails, a shared-expert group

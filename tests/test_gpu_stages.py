@@ -13,6 +13,10 @@ pytestmark = pytest.mark.gpu
 ROUTE_SHAPES = [
     I.WORKLOADS["tiny_T16"],
     I.MoEShape("cuda_core_router", 37, 256, 64, 64, 6, 6, zipf_s=0.8),     # E > 32, small T·E·d
+    # decode batches (T <= 8, E > 32): the one-kernel GEMV router
+    I.MoEShape("gemv_router_T5", 5, 256, 96, 64, 6, 6, zipf_s=1.0),
+    I.MoEShape("gemv_router_T1_E1000", 1, 512, 1000, 64, 8, 8),
+    I.MoEShape("gemv_router_elastic_T7", 7, 256, 64, 64, 2, 8, k_choices=(1, 2, 4, 8)),
     # the tensor-core router (T·E·d >= 2^29): E % 128 != 0 and T % 64 != 0, and E = 33
     I.MoEShape("mma_router_ragged_E", 1000, 1056, 520, 64, 4, 4),
     I.MoEShape("mma_router_E33", 8200, 2048, 33, 64, 3, 3),
