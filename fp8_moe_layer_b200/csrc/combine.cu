@@ -14,9 +14,9 @@
 namespace moe {
 
 // s2[r] = amax[r] / 448 (IEEE fp32; 1 if 0); aq[r, f] = e4m3_rne_satfinite(act[r, f] / s2[r]).
-// The row max is already complete (from the gate/up epilogue), so every 4-element chunk of every
-// row is independent: a 2-D grid (row stride x column chunk), so no thread divides its index,
-// 128-bit loads, 32-bit stores.
+// The row max is already complete (from the gate/up epilogue), so every 16-element chunk of every
+// row is independent: a 2-D grid (row stride x chunk), four 16-byte loads in flight per thread and
+// one 16-byte store, no thread divides its index.
 __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ act,
                                                       const uint32_t* __restrict__ amax,
                                                       const int32_t* __restrict__ total_rows,
@@ -25,20 +25,23 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
                                                       float* __restrict__ s2) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  // grid: x strides over rows, y over chunks of blockDim.x float4s of a row
   const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
-  const int nv = F / 4;
+  const int n16 = F / 16;
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
-  if (c >= nv) return;
-#pragma unroll 4
+  if (c >= n16) return;
+#pragma unroll 2
   for (int r = blockIdx.x; r < R; r += gridDim.x) {
     const float am = __uint_as_float(amax[r]);
     const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
     if (c == 0) s2[r] = sc;
-    const float4 v = reinterpret_cast<const float4*>(act + (size_t)r * F)[c];
-    reinterpret_cast<uint32_t*>(aq + (size_t)r * F)[c] =
-        static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.x, sc), __fdiv_rn(v.y, sc))) |
-        (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.z, sc), __fdiv_rn(v.w, sc))) << 16);
+    const float4* src = reinterpret_cast<const float4*>(act + (size_t)r * F) + 4 * c;
+    const float4 v[4] = {src[0], src[1], src[2], src[3]};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o[q] = static_cast<uint32_t>(e4m3x2(__fdiv_rn(v[q].x, sc), __fdiv_rn(v[q].y, sc))) |
+             (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v[q].z, sc), __fdiv_rn(v[q].w, sc))) << 16);
+    reinterpret_cast<uint4*>(aq + (size_t)r * F)[c] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -179,9 +182,9 @@ static int row_grid(int64_t rows) {
 
 cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
                            const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s) {
-  const int nv = p.F / 4;
-  const int threads = std::min(256, ((nv + 31) / 32) * 32);
-  const int gy = (nv + threads - 1) / threads;
+  const int n16 = p.F / 16;
+  const int threads = std::min(256, ((n16 + 31) / 32) * 32);
+  const int gy = (n16 + threads - 1) / threads;
   const int gx = (int)std::min<int64_t>(std::max<int64_t>(p.Rcap, 1),
                                         std::max<int64_t>(16LL * num_sms() / gy, 1));
   launch_pdl(requant_kernel, dim3(gx, gy), dim3(threads), 0, s, act, amax, total_rows, p.Rcap,

@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(
     const int t = s_perm[r];
     const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(xqp + (size_t)r * d);
+#pragma unroll 4
     for (int i = lane; i < nv; i += 32) dst[i] = src[i];
     if (lane == 0) {
       xsp[r] = xs[t];
@@ -394,6 +395,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(
     uint4* dst = reinterpret_cast<uint4*>(xqp + (size_t)r * d);
     if (ok) {
       const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
+#pragma unroll 4
       for (int i = lane; i < nv; i += 32) dst[i] = src[i];
     } else {
       for (int i = lane; i < nv; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
