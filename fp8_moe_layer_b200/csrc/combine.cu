@@ -15,8 +15,10 @@ namespace moe {
 
 // s2[r] = amax[r] / 448 (IEEE fp32; 1 if 0); aq[r, f] = e4m3_rne_satfinite(act[r, f] / s2[r]).
 // The row max is already complete (from the gate/up epilogue), so every 16-element chunk of every
-// row is independent: a 2-D grid (row stride x chunk), four 16-byte loads in flight per thread and
-// one 16-byte store, no thread divides its index.
+// row is independent: thread (x, y) of a (chunks x rows) block takes chunk blockIdx.y * blockDim.x
+// + x of rows blockIdx.x * blockDim.y + y, stepping by gridDim.x * blockDim.y (short rows fill the
+// block with several rows); four 16-byte loads in flight per thread and one 16-byte store, no
+// thread divides its index.
 __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ act,
                                                       const uint32_t* __restrict__ amax,
                                                       const int32_t* __restrict__ total_rows,
@@ -30,7 +32,7 @@ __global__ void __launch_bounds__(256) requant_kernel(const float* __restrict__ 
   const int c = blockIdx.y * blockDim.x + threadIdx.x;
   if (c >= n16) return;
 #pragma unroll 2
-  for (int r = blockIdx.x; r < R; r += gridDim.x) {
+  for (int r = blockIdx.x * blockDim.y + threadIdx.y; r < R; r += gridDim.x * blockDim.y) {
     const float am = __uint_as_float(amax[r]);
     const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
     if (c == 0) s2[r] = sc;
@@ -183,11 +185,13 @@ static int row_grid(int64_t rows) {
 cudaError_t launch_requant(const Plan& p, const float* act, const uint32_t* amax,
                            const int32_t* total_rows, uint8_t* aq, float* s2, cudaStream_t s) {
   const int n16 = p.F / 16;
-  const int threads = std::min(256, ((n16 + 31) / 32) * 32);
-  const int gy = (n16 + threads - 1) / threads;
-  const int gx = (int)std::min<int64_t>(std::max<int64_t>(p.Rcap, 1),
+  const int bx = std::min(256, n16);                 // chunks of a row per block
+  const int by = std::max(1, 256 / bx);              // rows per block
+  const int gy = (n16 + bx - 1) / bx;
+  const int64_t row_blocks = (p.Rcap + by - 1) / by;
+  const int gx = (int)std::min<int64_t>(std::max<int64_t>(row_blocks, 1),
                                         std::max<int64_t>(16LL * num_sms() / gy, 1));
-  launch_pdl(requant_kernel, dim3(gx, gy), dim3(threads), 0, s, act, amax, total_rows, p.Rcap,
+  launch_pdl(requant_kernel, dim3(gx, gy), dim3(bx, by), 0, s, act, amax, total_rows, p.Rcap,
              p.F, aq, s2);
   return cudaGetLastError();
 }
