@@ -71,7 +71,9 @@ typedef struct moe_dims {
  *     event i is recorded on `stream` just before stage i's kernel, the last one after the last
  *     stage. Stages: 0 router logits, 1 top-k + activation quantisation, 2 permutation,
  *     3 row gather, 4 gate/up GEMM + SwiGLU, 5 intermediate requantisation, 6 down GEMM,
- *     7 combine. */
+ *     7 combine. A stage computed by the previous stage's kernel brackets nothing: stage 1 when
+ *     one kernel routes and quantises (E <= 32, or decode batches of T <= 8), stage 3 when one
+ *     kernel groups and gathers the rows (T * k_max <= 8192). */
 #define MOE_NUM_STAGES 8
 typedef struct moe_debug_out {
   int32_t* topk_ids;
@@ -89,8 +91,10 @@ size_t moe_workspace_bytes(const moe_dims* dims);
 /* Host only, pure. A static English description of a moe_status value. */
 const char* moe_status_string(int status);
 
-/* Clears the device status word kept at the start of `ws` (async on `stream`). moe_forward clears
- * it itself; callers of the split entry points clear it once after allocating `ws`. */
+/* Clears the device status word kept at the start of `ws` (16 bytes: error code, where-code,
+ * detail, and the completion counter of the one-kernel decode router), async on `stream`.
+ * moe_forward clears it itself; callers of the split entry points clear it once after
+ * allocating `ws`. */
 int moe_clear_status(void* ws, void* stream);
 
 /* Reads the device status word of `ws` into *out_status (MOE_OK or a MOE_ERR_DEVICE_* code).
