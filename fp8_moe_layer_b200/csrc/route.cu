@@ -1,6 +1,12 @@
-// Router of the MoE layer: logits on CUDA cores (fp32 FMA, deterministic split over the hidden
-// dimension), then per token a warp-level softmax / top-k with renormalised weights, fused with
-// the token's dynamic FP8 e4m3 quantisation (scale = amax / 448).
+// Router of the MoE layer: logits, softmax / top-k with renormalised weights, and the token's
+// dynamic FP8 e4m3 quantisation (scale = amax / 448). Four kernels, by shape:
+//   route_block_kernel   E <= 32: one block per token does all of it;
+//   route_gemv_kernel    decode batches (T <= 8, E > 32): a warp per expert, and the last block
+//                        to finish selects and quantises;
+//   router_logits_kernel fp32 CUDA-core logits (deterministic split over the hidden dimension),
+//   + topk_quant_kernel  then per token a warp-level top-k and the quantisation;
+//   topk_quant_kernel    also after the tensor-core logits (router_mma.cu), refining the
+//                        candidates' logits exactly before the selection.
 //
 // Method: "Routage MoE entre GPU" (viite.ai) -- the router scores all experts from the hidden
 // state, keeps the top-k and emits one routing weight per selection; the megakernel page
