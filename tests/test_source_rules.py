@@ -35,3 +35,22 @@ def test_no_trap_or_device_assert():
         src = re.sub(r"//.*", "", open(path).read())
         src = src.replace("static_assert(", "")          # compile-time checks are fine
         assert "__trap" not in src and "trap;" not in src and "assert(" not in src, path
+
+
+def test_no_cluster_multicast_loads():
+    # The library runs as replicas on several GPUs; no load may use cluster multicast (the pair
+    # GEMM signals its two CTAs with separate commits instead). The qualifier is assembled here
+    # so that this file does not spell it.
+    qualifier = "." + "multicast" + "::" + "cluster"
+    for path in glob.glob(os.path.join(CSRC, "*.cu*")):
+        assert qualifier not in open(path).read(), path
+
+
+def test_every_spin_wait_is_bounded():
+    # mbarrier polls go through the bounded helpers only (a timeout records a status and returns)
+    for path in glob.glob(os.path.join(CSRC, "*.cu*")):
+        src = re.sub(r"//.*", "", open(path).read())
+        if os.path.basename(path) == "common.cuh":
+            continue                                    # the helpers themselves
+        assert "mbarrier.try_wait" not in src, path
+        assert "while (!mbar_try_wait" not in src and "while(!mbar_try_wait" not in src, path
