@@ -13,6 +13,11 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp8moe.so")
+# The wait-test build: the same sources with every in-kernel wait bounded at 2 ms and a host
+# switch that withholds one GEMM signal (include/moe_testing.h), for the tests of the
+# device-timeout path. Nothing but those tests loads it.
+LIB_WAITTEST = os.path.join(HERE, "libfp8moe_waittest.so")
+VARIANTS = {LIB: [], LIB_WAITTEST: ["-DMOE_WAIT_TEST"]}
 SOURCES = ["moe_api.cu", "route.cu", "router_mma.cu", "permute.cu", "gemm.cu", "combine.cu",
            "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -29,21 +34,25 @@ def sources():
     return [os.path.join(CSRC, s) for s in SOURCES]
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
-    deps.append(os.path.join(os.path.dirname(HERE), "include", "moe.h"))
+    inc = os.path.join(os.path.dirname(HERE), "include")
+    deps += [os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compile the library if any source is newer than it; returns its path."""
-    if not force and not needs_build():
-        return LIB
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          lib: str = LIB) -> str:
+    """Compile `lib` (the library, or its wait-test build) if any source is newer than it;
+    returns its path."""
+    if not force and not needs_build(lib):
+        return lib
     cmd = [nvcc_path(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-shared", "-cudart", "shared",
-           "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "-o", LIB + ".tmp", *sources()]
+           "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", *VARIANTS[lib], "-o", lib + ".tmp",
+           *sources()]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
@@ -53,10 +62,12 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose or ptxas_info:
         print(res.stdout + res.stderr, file=sys.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv)
-    print(LIB)
+    for target in ([LIB, LIB_WAITTEST] if "--all" in sys.argv else [LIB]):
+        build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv,
+              lib=target)
+        print(target)

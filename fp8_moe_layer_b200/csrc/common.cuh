@@ -9,9 +9,16 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace moe {
+
+// Kernels launched by this library in this process (every launch goes through launch_pdl*).
+inline std::atomic<unsigned long long>& launch_counter() {
+  static std::atomic<unsigned long long> n{0};
+  return n;
+}
 
 // ---------------------------------------------------------------- status word (lives in ws[0..3])
 constexpr int kStatusDeviceTimeout = -5;
@@ -32,7 +39,13 @@ __device__ __forceinline__ void report(int* status, int code, int where, int det
 }
 
 // Upper bound of every spin-wait: ~1 s of %globaltimer, and an iteration cap as a second bound.
+// The wait-test build (MOE_WAIT_TEST, a separate library used only by the tests of the timeout
+// path) bounds every wait at 2 ms instead.
+#ifdef MOE_WAIT_TEST
+constexpr uint64_t kWaitLimitNs = 2ull * 1000ull * 1000ull;
+#else
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+#endif
 constexpr uint32_t kWaitMaxIters = 1u << 26;
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -371,6 +384,7 @@ inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = cluster_x > 1 ? 2 : 1;
+  launch_counter().fetch_add(1, std::memory_order_relaxed);
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -387,6 +401,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  launch_counter().fetch_add(1, std::memory_order_relaxed);
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 

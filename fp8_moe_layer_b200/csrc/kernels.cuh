@@ -23,6 +23,7 @@ struct Plan {
   int64_t Rpad;      // rows allocated for row-indexed buffers (>= Rcap, >= 256)
   int BN;            // token tile of the grouped GEMMs (max MMA N; a tile uses its valid rows)
   bool pair1, pair2; // gate/up, down GEMM on 2-CTA pairs (M = 256 tcgen05 MMA)
+  int slabs1;        // weight slabs of 128 rows per CTA in the gate/up GEMM (2: pairs only)
   int r_splits, r_chunks_per_split;           // router: split of d into 32-wide chunks
   int g1_kb, g1_m_tiles;                      // gate/up GEMM: K blocks (d/128), 64-row tiles
   int g1_splits, g1_kb_per_split;             // gate/up K split (decode); 1 = SwiGLU epilogue
@@ -55,14 +56,33 @@ struct GemmArgs {
   size_t out_split_stride;       // elements between split partials
   uint32_t* row_amax;            // gate/up: [Rpad] |act| max as fp32 bits
   int* status;
+#ifdef MOE_WAIT_TEST
+  int withhold;                  // wait-test build: skip the first tile's accumulator signal
+#endif
 };
+
+#ifdef MOE_WAIT_TEST
+// Wait-test build only: when set, every CTA of the next gate/up GEMMs withholds the "accumulator
+// ready" signal of its first tile, so that the epilogue's bounded wait expires.
+extern int g_withhold_gemm_commit;
+#endif
+
+// Planning assumes the B200's 148 SMs so that moe_workspace_bytes stays a pure host function;
+// persistent grids use the real SM count of the current device.
+constexpr int kPlanSMs = 148;
+
+// The CUDA-core router logits kernel's cut of d: 32-token x 32-expert tiles and enough pieces of
+// d (each `*chunks_per_split` 32-wide chunks) for about two waves of kPlanSMs; returns the number
+// of pieces (the splits of the partial logits).
+int router_splits(int T, int d, int E, int* chunks_per_split);
 
 // k_est: experts per token the GEMM tiles are planned for (0 = k_max); buffers are for k_max.
 int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est = 0);
 
+// Router logits are fp64 (part [splits][T][E] doubles): see route.cu.
 cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
-                                 float* part, cudaStream_t s);
-cudaError_t launch_topk_quant(const Plan& p, const float* part, const float* bias, int k,
+                                 double* part, cudaStream_t s);
+cudaError_t launch_topk_quant(const Plan& p, const double* part, const float* bias, int k,
                               const int32_t* k_per_token, int32_t* ids, float* w,
                               const uint16_t* hidden, uint8_t* xq, float* xs, bool do_route,
                               bool do_quant, const float* refine_w, int* status, cudaStream_t s);
@@ -87,12 +107,12 @@ inline bool router_uses_gemv(int E, int T, int d) {
 }
 inline bool router_uses_gemv(const Plan& p) { return router_uses_gemv(p.E, p.T, p.d); }
 cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
-                              const float* bias, int k, const int32_t* k_per_token, float* logits,
-                              int32_t* ids, float* w, uint8_t* xq, float* xs, bool do_quant,
-                              int* status, cudaStream_t s);
+                              const float* bias, int k, const int32_t* k_per_token,
+                              double* logits, int32_t* ids, float* w, uint8_t* xq, float* xs,
+                              bool do_quant, int* status, cudaStream_t s);
 // planes: 3 * E * d bf16 (workspace); map_w over planes [3][E][d], map_x over hidden [T][d]
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
-                              const CUtensorMap& map_w, const CUtensorMap& map_x, float* logits,
+                              const CUtensorMap& map_w, const CUtensorMap& map_x, double* logits,
                               int* status, cudaStream_t s);
 cudaError_t launch_route_fused(const Plan& p, const uint16_t* hidden, const float* router_w,
                                const float* bias, int k, const int32_t* k_per_token,

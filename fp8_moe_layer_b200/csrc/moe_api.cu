@@ -11,12 +11,12 @@
 
 namespace moe {
 
-// Planning assumes the B200's 148 SMs so that moe_workspace_bytes stays a pure host function;
-// persistent grids use the real SM count of the current device.
-constexpr int kPlanSMs = 148;
-
 static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+#ifdef MOE_WAIT_TEST
+int g_withhold_gemm_commit = 0;
+#endif
 
 int num_sms() {
   static int cache[64] = {};
@@ -49,6 +49,14 @@ static int choose_splits(int64_t base_tiles, int num_kb, int units, double w_til
     }
   }
   return best;
+}
+
+int router_splits(int T, int d, int E, int* chunks_per_split) {
+  const int64_t rtiles = ceil_div(std::max(T, 1), kRouterTile) * ceil_div(E, kRouterTile);
+  const int nchunks = (int)ceil_div(d, kRouterTile);
+  const int rs = (int)std::min<int64_t>(nchunks, std::max<int64_t>(1, ceil_div(2 * kPlanSMs, rtiles)));
+  *chunks_per_split = (int)ceil_div(nchunks, rs);
+  return (int)ceil_div(nchunks, *chunks_per_split);
 }
 
 int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est) {
@@ -91,14 +99,22 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
 #ifdef MOE_FORCE_PAIR
   p->pair1 = p->pair2 = MOE_FORCE_PAIR;
 #endif
+  // A prefill gate/up CTA holds two 128-row weight slabs against one token tile (two TMEM
+  // accumulators): the token rows cross L2 -> shared memory once per 512 weight rows of a pair,
+  // a quarter fewer bytes per MMA than one slab.
+  p->slabs1 = p->pair1 ? 2 : 1;
+#ifdef MOE_FORCE_SLABS
+  p->slabs1 = p->pair1 ? MOE_FORCE_SLABS : 1;
+#endif
 
-  // router: 32x32 tiles; split d so that the grid covers about two waves
-  const int64_t rtiles = ceil_div(std::max(T, 1), kRouterTile) * ceil_div(E, kRouterTile);
-  const int nchunks = (int)ceil_div(d, kRouterTile);
-  int rs = (int)std::min<int64_t>(nchunks, std::max<int64_t>(1, ceil_div(2 * kPlanSMs, rtiles)));
-  if (router_uses_mma(E, T, d)) rs = 1;      // the tensor-core router writes whole logits
-  p->r_chunks_per_split = (int)ceil_div(nchunks, rs);
-  p->r_splits = (int)ceil_div(nchunks, p->r_chunks_per_split);
+  // router: 32x32 tiles; split d so that the grid covers about two waves (the tensor-core router
+  // writes whole logits)
+  if (router_uses_mma(E, T, d)) {
+    p->r_splits = 1;
+    p->r_chunks_per_split = (int)ceil_div(d, kRouterTile);
+  } else {
+    p->r_splits = router_splits(T, d, E, &p->r_chunks_per_split);
+  }
 
   p->g1_kb = (int)ceil_div(d, kBK);
   p->g1_m_tiles = (int)ceil_div(F, 64);
@@ -127,7 +143,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + std::max<size_t>(bytes, 1)); return o; };
   p->off_status = take(256);
-  p->off_part = take(sizeof(float) * (size_t)p->r_splits * T * E);
+  p->off_part = take(sizeof(double) * (size_t)p->r_splits * T * E);
   p->off_ids = take(sizeof(int32_t) * (size_t)routed);
   p->off_w = take(sizeof(float) * (size_t)routed);
   p->off_offsets = take(sizeof(int32_t) * (size_t)(E + 2));
@@ -255,7 +271,8 @@ static int check_device() {
 
 struct Ws {
   int* status;
-  float *part, *w, *xs, *xsp, *act, *s2, *o, *hpart;
+  double* part;
+  float *w, *xs, *xsp, *act, *s2, *o, *hpart;
   uint16_t* planes;
   int32_t *ids, *offsets, *tiles, *perm, *inv, *pscr;
   uint8_t *xq, *xqp, *aq;
@@ -266,7 +283,7 @@ static Ws carve(const Plan& p, void* ws) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   Ws w;
   w.status = reinterpret_cast<int*>(b + p.off_status);
-  w.part = reinterpret_cast<float*>(b + p.off_part);
+  w.part = reinterpret_cast<double*>(b + p.off_part);
   w.ids = reinterpret_cast<int32_t*>(b + p.off_ids);
   w.w = reinterpret_cast<float*>(b + p.off_w);
   w.offsets = reinterpret_cast<int32_t*>(b + p.off_offsets);
@@ -368,6 +385,9 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g1.out_split_stride = 0;
   g1.row_amax = w.amax;
   g1.status = w.status;
+#ifdef MOE_WAIT_TEST
+  g1.withhold = g_withhold_gemm_commit;
+#endif
   const bool split1 = p.g1_splits > 1;
   if (split1) {
     g1.splits = p.g1_splits;
@@ -401,6 +421,9 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g2.out_ld = p.d;
   g2.out_split_stride = split_stride;
   g2.row_amax = nullptr;
+#ifdef MOE_WAIT_TEST
+  g2.withhold = 0;
+#endif
   // the down GEMM's TMA stores: o as [splits x split rows][d] fp32 (a caller's unsplit buffer
   // has exactly o_rows rows)
   CUtensorMap mo;
@@ -444,6 +467,14 @@ const char* moe_status_string(int status) {
     default: return "unknown status";
   }
 }
+
+uint64_t moe_kernel_launch_count(void) {
+  return static_cast<uint64_t>(launch_counter().load(std::memory_order_relaxed));
+}
+
+#ifdef MOE_WAIT_TEST
+void moe_test_withhold_gemm_commit(int on) { g_withhold_gemm_commit = on ? 1 : 0; }
+#endif
 
 int moe_clear_status(void* ws, void* stream) {
   if (!ws) return MOE_ERR_WORKSPACE;

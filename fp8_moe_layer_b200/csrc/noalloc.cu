@@ -12,6 +12,7 @@
 // stand-in, so the kernels get its device address from cudaGetSymbolAddress, taken once per
 // device (with that device current) by the first call on that device.
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 
 #include "../../include/moe.h"
@@ -24,20 +25,22 @@ static __device__ __align__(256) unsigned char g_route_scratch[MOE_NOALLOC_SCRAT
 
 namespace {
 constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
+// One cached address per device. Host threads that make their first call on a device at the same
+// time may both look it up; they store the same value, so relaxed atomics suffice.
+std::atomic<void*> g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_route_scratch on the current device (looked up once per device).
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
+  void* p = g_scratch_addr[dev].load(std::memory_order_relaxed);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
       return MOE_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    g_scratch_addr[dev].store(p, std::memory_order_relaxed);
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return MOE_OK;
 }
 }  // namespace
@@ -61,18 +64,12 @@ extern "C" int moe_route_topk_noalloc(const moe_dims* dims, const uint16_t* hidd
   if (k_per_token ? (reinterpret_cast<uintptr_t>(k_per_token) % 4) != 0
                   : (k < 1 || k > std::min(p.E, p.k_max)))
     return MOE_ERR_INVALID_ARG;
-  // Scratch: the partial logits of the CUDA-core router (the fused small-E router needs none).
+  // Scratch: the fp64 partial logits of the CUDA-core router (the fused small-E router needs
+  // none), cut into pieces of d the same way as the workspace router's CUDA-core path
   const bool fused = router_is_fused(p);
-  // the CUDA-core logits kernel's cut of d: 32x32 (token x expert) tiles, enough pieces of d for
-  // about two waves of 148 SMs
-  const long long rtiles = ((std::max(p.T, 1) + kRouterTile - 1) / kRouterTile) *
-                           (long long)((p.E + kRouterTile - 1) / kRouterTile);
-  const int nchunks = (p.d + kRouterTile - 1) / kRouterTile;
-  const int want = (int)std::max(1LL, (2LL * 148 + rtiles - 1) / rtiles);
-  const int cut = std::min(nchunks, want);
-  const int chunks = (nchunks + cut - 1) / cut;
-  const int splits = (nchunks + chunks - 1) / chunks;
-  const size_t need = fused ? 0 : sizeof(float) * (size_t)splits * p.T * p.E;
+  int chunks = 0;
+  const int splits = router_splits(p.T, p.d, p.E, &chunks);
+  const size_t need = fused ? 0 : sizeof(double) * (size_t)splits * p.T * p.E;
   if (need > MOE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int major = 0, dev = 0;
@@ -93,7 +90,7 @@ extern "C" int moe_route_topk_noalloc(const moe_dims* dims, const uint16_t* hidd
   Plan q = p;                      // always the CUDA-core logits (no tensor-core weight planes)
   q.r_splits = splits;
   q.r_chunks_per_split = chunks;
-  float* part = static_cast<float*>(scratch);
+  double* part = static_cast<double*>(scratch);
   if (launch_router_logits(q, hidden, router_w, part, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (launch_topk_quant(q, part, router_bias, k, k_per_token, topk_ids, topk_w, hidden, nullptr,
                         nullptr, true, false, nullptr, nullptr, s) != cudaSuccess)

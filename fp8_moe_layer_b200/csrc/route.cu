@@ -11,30 +11,107 @@
 // Method: "Routage MoE entre GPU" (viite.ai) -- the router scores all experts from the hidden
 // state, keeps the top-k and emits one routing weight per selection; the megakernel page
 // (seventnews.com), W8A8 paragraph -- 8-bit FP8 activations.
+//
+// Precision of the routing decision: a bf16 hidden value times an fp32 router weight is exact in
+// fp64 (8 + 24 significand bits), so every logit that decides a selection is summed in fp64. The
+// selection and the slot order then agree with an fp64 evaluation of the same dot products except
+// where two logits lie within the fp64 summation error (~1e-12 at d = 7168) of each other. The
+// tensor-core logits (router_mma.cu) are only a filter: the experts they leave in play are
+// recomputed in fp64 before the selection. The weights exp(l_j - l_max) / sum are computed in fp64
+// and rounded once to fp32.
 #include "common.cuh"
 #include "kernels.cuh"
 
 namespace moe {
 
-// part[s][t][e] = sum over the d-chunks of split s of x[t, d] * W[e, d], fp32, d ascending,
-// one partial sum per 32-wide chunk (blocked summation keeps the rounding error near fp64).
+// Warp-wide selection of the kt largest of n values, descending, exact ties to the lower id:
+// candidate slot c (c = lane, lane + 32, ...; n <= 1024) has value val(c) and id idf(c). Lane j < kt
+// receives the j-th selected (value, id).
+template <typename ValFn, typename IdFn>
+__device__ __forceinline__ void warp_select_desc(int n, int kt, ValFn val, IdFn idf, double& sel_v,
+                                                 int& sel_e) {
+  const int lane = threadIdx.x & 31;
+  uint32_t taken = 0;            // bit i: slot lane + 32 i already selected
+  sel_v = 0.0;
+  sel_e = -1;
+  for (int j = 0; j < kt; ++j) {
+    double bv = -INFINITY;
+    int be = 0x7FFFFFFF, bslot = -1;
+    for (int i = 0, c = lane; c < n; ++i, c += 32) {
+      const double v = val(c);
+      const int e = idf(c);
+      if (!((taken >> i) & 1u) && (v > bv || (v == bv && e < be))) {
+        bv = v;
+        be = e;
+        bslot = c;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      const int os = __shfl_xor_sync(0xffffffffu, bslot, off);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+        bslot = os;
+      }
+    }
+    if (bslot >= 0 && (bslot & 31) == lane) taken |= 1u << (bslot >> 5);
+    if (lane == j) {
+      sel_v = bv;
+      sel_e = be;
+    }
+  }
+}
+
+// Renormalised weights of the selection held by lanes j < kt (sel_v descending): fp64
+// exp(l_j - l_max) / sum, rounded once to fp32; ids and weights of slots >= kt are -1 and 0.
+__device__ __forceinline__ void warp_store_selection(double sel_v, int sel_e, int kt, int k_max,
+                                                     int32_t* ids, float* wout) {
+  const int lane = threadIdx.x & 31;
+  const double lmax = __shfl_sync(0xffffffffu, sel_v, 0);
+  const double z = lane < kt ? exp(sel_v - lmax) : 0.0;
+  double zs = z;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
+  if (lane < k_max) {
+    ids[lane] = lane < kt ? sel_e : -1;
+    wout[lane] = lane < kt ? static_cast<float>(z / zs) : 0.f;
+  }
+}
+
+// fp64 dot product of 8 bf16 values (packed in v) with 8 fp32 weights (a, b): each product is exact.
+__device__ __forceinline__ double dot8_f64(const uint4 v, const float4 a, const float4 b) {
+  double c = static_cast<double>(__uint_as_float(v.x << 16)) * a.x;
+  c = fma(static_cast<double>(__uint_as_float(v.x & 0xFFFF0000u)), static_cast<double>(a.y), c);
+  c = fma(static_cast<double>(__uint_as_float(v.y << 16)), static_cast<double>(a.z), c);
+  c = fma(static_cast<double>(__uint_as_float(v.y & 0xFFFF0000u)), static_cast<double>(a.w), c);
+  c = fma(static_cast<double>(__uint_as_float(v.z << 16)), static_cast<double>(b.x), c);
+  c = fma(static_cast<double>(__uint_as_float(v.z & 0xFFFF0000u)), static_cast<double>(b.y), c);
+  c = fma(static_cast<double>(__uint_as_float(v.w << 16)), static_cast<double>(b.z), c);
+  c = fma(static_cast<double>(__uint_as_float(v.w & 0xFFFF0000u)), static_cast<double>(b.w), c);
+  return c;
+}
+
+// part[s][t][e] = sum over the d-chunks of split s of x[t, d] * W[e, d], fp64, d ascending.
 // Block: 256 threads computing a 32-token x 32-expert tile; thread (ty, tx) owns tokens
-// 4*ty .. 4*ty+3 of expert tx.
+// 4*ty .. 4*ty+3 of expert tx. The tiles hold the inputs as fp64 (exact conversions).
 __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
                                                             const float* __restrict__ W, int T,
                                                             int d, int E, int chunks_per_split,
-                                                            float* __restrict__ part) {
+                                                            double* __restrict__ part) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  __shared__ float xs[kRouterTile][kRouterTile + 1];
-  __shared__ float ws[kRouterTile][kRouterTile + 1];
+  __shared__ double xs[kRouterTile][kRouterTile + 1];
+  __shared__ double ws[kRouterTile][kRouterTile + 1];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int t0 = blockIdx.x * kRouterTile, e0 = blockIdx.y * kRouterTile;
   const int split = blockIdx.z;
   const int nchunks = (d + kRouterTile - 1) / kRouterTile;
   const int c_begin = split * chunks_per_split;
   const int c_end = min(nchunks, c_begin + chunks_per_split);
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
   for (int c = c_begin; c < c_end; ++c) {
     const int dbase = c * kRouterTile;
 #pragma unroll
@@ -42,20 +119,16 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
       const int r = ty + 8 * i;            // row of the tile this thread loads
       const int dd = dbase + tx;
       const int t = t0 + r, e = e0 + r;
-      xs[r][tx] = (t < T && dd < d) ? bf16_bits_to_float(x[(size_t)t * d + dd]) : 0.f;
-      ws[r][tx] = (e < E && dd < d) ? W[(size_t)e * d + dd] : 0.f;
+      xs[r][tx] = (t < T && dd < d) ? static_cast<double>(bf16_bits_to_float(x[(size_t)t * d + dd])) : 0.0;
+      ws[r][tx] = (e < E && dd < d) ? static_cast<double>(W[(size_t)e * d + dd]) : 0.0;
     }
     __syncthreads();
-    // blocked summation: each 32-wide chunk is summed on its own, then added to the total
-    float chunk[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
     for (int kk = 0; kk < kRouterTile; ++kk) {
-      const float w = ws[tx][kk];
+      const double w = ws[tx][kk];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) chunk[i] = fmaf(xs[4 * ty + i][kk], w, chunk[i]);
+      for (int i = 0; i < 4; ++i) acc[i] = fma(xs[4 * ty + i][kk], w, acc[i]);
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i] += chunk[i];
     __syncthreads();
   }
   const int e = e0 + tx;
@@ -69,29 +142,33 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 }
 
 // One block (128 threads) per token.
-//  route: l[e] = sum_s part[s][t][e] + bias[e]; k_t largest (descending, exact ties to the lower
-//         expert id); w_j = exp(l_j - l_max) / sum_sel exp(l_sel - l_max), which equals the
-//         softmax over all E renormalised over the selection.
+//  route: l[e] = sum_s part[s][t][e] + bias[e] (fp64, splits in fixed order); the k_t largest
+//         (descending, exact ties to the lower expert id) and their renormalised weights
+//         exp(l_j - l_max) / sum_sel exp(l_sel - l_max), which equal the softmax over all E
+//         renormalised over the selection.
 //  quant: s_t = amax|x[t,:]| / 448 (IEEE fp32 division; 1 if amax = 0);
 //         xq = e4m3_rne_satfinite(x / s_t) (IEEE fp32 division).
 //  refine (refine_w != null, for the tensor-core logits): the approximate logits only pick the
 //         candidates -- every expert within kRefineWindow of the approximate k_t-th largest, which
 //         contains the exact top-k_t while the approximation error stays below half the window --
-//         and each candidate's logit is recomputed exactly (fp32, one warp per candidate, fixed
-//         order) before the selection and the weights.
-constexpr float kRefineWindow = 1e-2f;
+//         and each candidate's logit is recomputed in fp64 (one warp per candidate) before the
+//         selection and the weights.
+constexpr double kRefineWindow = 1e-2;
 constexpr int kMaxCandidates = 256;
 
 __global__ void __launch_bounds__(128) topk_quant_kernel(
-    const float* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E,
+    const double* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E,
     int k, const int32_t* __restrict__ k_per_token, int k_max, int32_t* __restrict__ ids,
     float* __restrict__ wout, const uint16_t* __restrict__ x, int d, uint8_t* __restrict__ xq,
     float* __restrict__ xs, int do_route, int do_quant, const float* __restrict__ refine_w,
     int* status) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  __shared__ float lg[kMaxExperts];
+  __shared__ double lg[kMaxExperts];
   __shared__ float red[4];
+  __shared__ int cand[kMaxCandidates];
+  __shared__ int ncand;
+  __shared__ double vk_s;
   const int t = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -99,15 +176,15 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
     for (int e = tid; e < E; e += 128) {
       // split partials in fixed order: eight independent accumulators keep eight loads in
       // flight (a decode batch splits d finely, and these loads are the kernel's latency)
-      float a8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      double a8[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
       int s = 0;
       for (; s + 8 <= splits; s += 8) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) a8[u] += part[((size_t)(s + u) * T + t) * E + e];
       }
       for (int u = 0; s < splits; ++s, ++u) a8[u] += part[((size_t)s * T + t) * E + e];
-      float v = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
-      if (bias) v += bias[e];
+      double v = ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+      if (bias) v += static_cast<double>(bias[e]);
       lg[e] = v;
     }
     __syncthreads();
@@ -117,49 +194,24 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
       if (tid == 0) report(status, kStatusDeviceCheck, kWhereRoute, t);
       kt = max(1, min(kt, kcap));
     }
-    __shared__ int cand[kMaxCandidates];
-    __shared__ int ncand;
     bool by_cand = false;          // exact selection over the refined candidates only
     if (refine_w) {
-      __shared__ float vk_s;
       if (warp == 0) {
-        // approximate k_t-th largest logit
-        uint32_t taken = 0;
-        float bv = -INFINITY;
-        for (int j = 0; j < kt; ++j) {
-          bv = -INFINITY;
-          int be = 0x7FFFFFFF;
-          for (int i = 0, e = lane; e < E; ++i, e += 32) {
-            const float v = lg[e];
-            if (!((taken >> i) & 1u) && (v > bv || (v == bv && e < be))) {
-              bv = v;
-              be = e;
-            }
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (ov > bv || (ov == bv && oe < be)) {
-              bv = ov;
-              be = oe;
-            }
-          }
-          if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        }
+        double sv;
+        int se;
+        warp_select_desc(E, kt, [&](int c) { return lg[c]; }, [](int c) { return c; }, sv, se);
+        const double vk = __shfl_sync(0xffffffffu, sv, kt - 1);   // approximate k_t-th largest
         if (lane == 0) {
-          vk_s = bv;
+          vk_s = vk;
           ncand = 0;
         }
       }
       __syncthreads();
-      const float floor_v = vk_s - kRefineWindow;
+      const double floor_v = vk_s - kRefineWindow;
       for (int e = tid; e < E; e += 128) {
         if (lg[e] >= floor_v) {
           const int c = atomicAdd(&ncand, 1);
           if (c < kMaxCandidates) cand[c] = e;
-        } else {
-          lg[e] = -INFINITY;                            // out of the selection
         }
       }
       __syncthreads();
@@ -170,75 +222,25 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
       for (int c = warp; c < nc; c += 4) {
         const int e = all ? c : cand[c];
         const float4* wr = reinterpret_cast<const float4*>(refine_w + (size_t)e * d);
-        float acc = 0.f;
-#pragma unroll 8
-        for (int i = lane; i < nv; i += 32) {
-          const uint4 v = xr[i];
-          const float4 a = __ldg(wr + 2 * i), b = __ldg(wr + 2 * i + 1);
-          float c8 = __uint_as_float(v.x << 16) * a.x;
-          c8 = fmaf(__uint_as_float(v.x & 0xFFFF0000u), a.y, c8);
-          c8 = fmaf(__uint_as_float(v.y << 16), a.z, c8);
-          c8 = fmaf(__uint_as_float(v.y & 0xFFFF0000u), a.w, c8);
-          c8 = fmaf(__uint_as_float(v.z << 16), b.x, c8);
-          c8 = fmaf(__uint_as_float(v.z & 0xFFFF0000u), b.y, c8);
-          c8 = fmaf(__uint_as_float(v.w << 16), b.z, c8);
-          c8 = fmaf(__uint_as_float(v.w & 0xFFFF0000u), b.w, c8);
-          acc += c8;
-        }
+        double acc = 0.0;
+#pragma unroll 4
+        for (int i = lane; i < nv; i += 32) acc += dot8_f64(xr[i], __ldg(wr + 2 * i), __ldg(wr + 2 * i + 1));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) lg[e] = acc + (bias ? bias[e] : 0.f);
+        if (lane == 0) lg[e] = acc + (bias ? static_cast<double>(bias[e]) : 0.0);
       }
       __syncthreads();
       by_cand = !all;
     }
     if (warp == 0) {
-      // bit i of `taken`: scan slot lane + 32 i already selected (slot = expert, or candidate
-      // index when the refined candidates are scanned; the others hold -inf then)
-      uint32_t taken = 0;
-      float sel_v = 0.f;             // lane j keeps the j-th selected logit
-      int sel_e = -1;
-      const int n_scan = by_cand ? ncand : E;
-      for (int j = 0; j < kt; ++j) {
-        float bv = -INFINITY;
-        int be = 0x7FFFFFFF;
-        for (int i = 0, c = lane; c < n_scan; ++i, c += 32) {
-          const int e = by_cand ? cand[c] : c;
-          const float v = lg[e];
-          if (!((taken >> i) & 1u) && (v > bv || (v == bv && e < be))) {
-            bv = v;
-            be = e;
-          }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-          if (ov > bv || (ov == bv && oe < be)) {
-            bv = ov;
-            be = oe;
-          }
-        }
-        if (by_cand) {
-          for (int i = 0, c = lane; c < n_scan; ++i, c += 32)
-            if (cand[c] == be) taken |= 1u << i;
-        } else if ((be & 31) == lane) {
-          taken |= 1u << (be >> 5);
-        }
-        if (lane == j) {
-          sel_v = bv;
-          sel_e = be;
-        }
-      }
-      const float lmax = __shfl_sync(0xffffffffu, sel_v, 0);
-      const float z = lane < kt ? expf(sel_v - lmax) : 0.f;
-      float zs = z;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
-      if (lane < k_max) {
-        ids[(size_t)t * k_max + lane] = lane < kt ? sel_e : -1;
-        wout[(size_t)t * k_max + lane] = lane < kt ? z / zs : 0.f;
-      }
+      double sv;
+      int se;
+      if (by_cand)
+        warp_select_desc(ncand, kt, [&](int c) { return lg[cand[c]]; },
+                         [&](int c) { return cand[c]; }, sv, se);
+      else
+        warp_select_desc(E, kt, [&](int c) { return lg[c]; }, [](int c) { return c; }, sv, se);
+      warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
     }
   }
 
@@ -281,58 +283,47 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
   }
 }
 
-// Decode router (T <= 8 tokens, E > 32): one warp per expert computes that expert's logit for
-// every token (lane-strided chunks of 8 along d, fp32, then a butterfly; all loads in flight),
+// Decode router (T <= 8 tokens, E > 32): one warp per expert computes that expert's fp64 logit
+// for every token (lane-strided chunks of 8 along d, then a butterfly; all loads in flight),
 // writes it to `logits` [T][E], and the last block to finish (a counter in the status word,
 // status[3]) selects the top-k, the weights and the FP8 quantisation of every token, then resets
 // the counter. One kernel instead of the tiled logits kernel (one global round trip per 32-wide
-// chunk of d) plus a separate top-k kernel.
+// chunk of d) plus a separate top-k kernel. Dynamic shared memory: T * E doubles (the last
+// block's copy of the logits).
 constexpr int kGemvMaxT = 8;
 
 template <int TT>
 __global__ void __launch_bounds__(256) route_gemv_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ W, const float* __restrict__ bias,
     int T, int d, int E, int k, const int32_t* __restrict__ k_per_token, int k_max,
-    float* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
+    double* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
     uint8_t* __restrict__ xq, float* __restrict__ xs, int do_quant, int* status) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   __shared__ int s_last;
-  __shared__ float lg[kGemvMaxT][kMaxExperts];
+  extern __shared__ double lgd[];                 // [T][E], used by the last block only
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int e = blockIdx.x * 8 + warp;
   const int nv = d / 8;
   if (e < E) {
-    float acc[TT];
+    double acc[TT];
 #pragma unroll
-    for (int j = 0; j < TT; ++j) acc[j] = 0.f;
+    for (int j = 0; j < TT; ++j) acc[j] = 0.0;
     const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
 #pragma unroll 4
     for (int i = lane; i < nv; i += 32) {
       const float4 a = __ldg(wr + 2 * i), b = __ldg(wr + 2 * i + 1);
 #pragma unroll
-      for (int j = 0; j < TT; ++j) {
-        if (j < T) {
-          const uint4 v = reinterpret_cast<const uint4*>(x + (size_t)j * d)[i];
-          float c8 = __uint_as_float(v.x << 16) * a.x;
-          c8 = fmaf(__uint_as_float(v.x & 0xFFFF0000u), a.y, c8);
-          c8 = fmaf(__uint_as_float(v.y << 16), a.z, c8);
-          c8 = fmaf(__uint_as_float(v.y & 0xFFFF0000u), a.w, c8);
-          c8 = fmaf(__uint_as_float(v.z << 16), b.x, c8);
-          c8 = fmaf(__uint_as_float(v.z & 0xFFFF0000u), b.y, c8);
-          c8 = fmaf(__uint_as_float(v.w << 16), b.z, c8);
-          c8 = fmaf(__uint_as_float(v.w & 0xFFFF0000u), b.w, c8);
-          acc[j] += c8;
-        }
-      }
+      for (int j = 0; j < TT; ++j)
+        if (j < T) acc[j] += dot8_f64(reinterpret_cast<const uint4*>(x + (size_t)j * d)[i], a, b);
     }
 #pragma unroll
     for (int j = 0; j < TT; ++j) {
       if (j < T) {
-        float v = acc[j];
+        double v = acc[j];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) logits[(size_t)j * E + e] = v + (bias ? bias[e] : 0.f);
+        if (lane == 0) logits[(size_t)j * E + e] = v + (bias ? static_cast<double>(bias[e]) : 0.0);
       }
     }
   }
@@ -345,7 +336,7 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
   __threadfence();
   if (warp < T) {
     const int t = warp;
-    float* my = lg[warp];
+    double* my = lgd + (size_t)t * E;
     for (int ee = lane; ee < E; ee += 32) my[ee] = __ldcg(logits + (size_t)t * E + ee);
     __syncwarp();
     int kt = k_per_token ? k_per_token[t] : k;
@@ -354,43 +345,10 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
       if (lane == 0) report(status, kStatusDeviceCheck, kWhereRoute, t);
       kt = max(1, min(kt, kcap));
     }
-    uint32_t taken = 0;            // bit i: expert lane + 32*i already selected
-    float sel_v = 0.f;             // lane j keeps the j-th selected logit
-    int sel_e = -1;
-    for (int j = 0; j < kt; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7FFFFFFF;
-      for (int i = 0, ee = lane; ee < E; ++i, ee += 32) {
-        const float v = my[ee];
-        if (!((taken >> i) & 1u) && (v > bv || (v == bv && ee < be))) {
-          bv = v;
-          be = ee;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == j) {
-        sel_v = bv;
-        sel_e = be;
-      }
-    }
-    const float lmax = __shfl_sync(0xffffffffu, sel_v, 0);
-    const float z = lane < kt ? expf(sel_v - lmax) : 0.f;
-    float zs = z;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
-    if (lane < k_max) {
-      ids[(size_t)t * k_max + lane] = lane < kt ? sel_e : -1;
-      wout[(size_t)t * k_max + lane] = lane < kt ? z / zs : 0.f;
-    }
+    double sv;
+    int se;
+    warp_select_desc(E, kt, [&](int c) { return my[c]; }, [](int c) { return c; }, sv, se);
+    warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
   }
   if (do_quant) {
     // the FP8 quantisation of each token by the whole block
@@ -441,7 +399,7 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
 
 // Small-E router (E <= 32), one 256-thread block per token, fully fused: logits, top-k, weights
 // and the token's FP8 quantisation. Thread i accumulates x[t, 8c..8c+7] . W[e, 8c..8c+7] for the
-// chunks c = i, i + 256, ... (fp32), a butterfly inside each warp and a fixed-order sum over the
+// chunks c = i, i + 256, ... in fp64, a butterfly inside each warp and a fixed-order sum over the
 // 8 warps complete each logit (deterministic), and lane e of warp 0 owns expert e's logit for the
 // selection. The row amax comes from the same pass and the chunks stay in registers for the
 // quantisation.
@@ -454,15 +412,15 @@ __global__ void __launch_bounds__(256) route_block_kernel(
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   constexpr int kChunks = 4;                      // d <= 256 * 8 * kChunks = 8192
-  __shared__ float part[8][EP];
+  __shared__ double part[8][EP];
   __shared__ float red[8];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = blockIdx.x;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
   const int nv = d / 8;
-  float acc[EP];
+  double acc[EP];
 #pragma unroll
-  for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+  for (int e = 0; e < EP; ++e) acc[e] = 0.0;
   uint4 xv[kChunks];
   float amax = 0.f;
 #pragma unroll
@@ -471,34 +429,22 @@ __global__ void __launch_bounds__(256) route_block_kernel(
     if (i < nv) {
       xv[c] = xr[i];
       const uint32_t w4[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
-      float xf[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        xf[2 * q] = __uint_as_float(w4[q] << 16);
-        xf[2 * q + 1] = __uint_as_float(w4[q] & 0xFFFF0000u);
-        amax = fmaxf(amax, fmaxf(fabsf(xf[2 * q]), fabsf(xf[2 * q + 1])));
-      }
+      for (int q = 0; q < 4; ++q)
+        amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[q] << 16)),
+                                 fabsf(__uint_as_float(w4[q] & 0xFFFF0000u))));
 #pragma unroll
       for (int e = 0; e < EP; ++e) {
         if (e < E) {
           const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d) + 2 * i;
-          const float4 a = __ldg(wr), b = __ldg(wr + 1);
-          float v = xf[0] * a.x;
-          v = fmaf(xf[1], a.y, v);
-          v = fmaf(xf[2], a.z, v);
-          v = fmaf(xf[3], a.w, v);
-          v = fmaf(xf[4], b.x, v);
-          v = fmaf(xf[5], b.y, v);
-          v = fmaf(xf[6], b.z, v);
-          v = fmaf(xf[7], b.w, v);
-          acc[e] += v;
+          acc[e] += dot8_f64(xv[c], __ldg(wr), __ldg(wr + 1));
         }
       }
     }
   }
 #pragma unroll
   for (int e = 0; e < EP; ++e) {
-    float v = acc[e];
+    double v = acc[e];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
     if (lane == 0) part[warp][e] = v;
@@ -509,12 +455,12 @@ __global__ void __launch_bounds__(256) route_block_kernel(
   __syncthreads();
 
   if (warp == 0) {
-    float logit = -INFINITY;
+    double logit = -INFINITY;
     if (lane < E) {
-      float v = 0.f;
+      double v = 0.0;
 #pragma unroll
       for (int w = 0; w < 8; ++w) v += part[w][lane < EP ? lane : 0];
-      logit = v + (bias ? bias[lane] : 0.f);
+      logit = v + (bias ? static_cast<double>(bias[lane]) : 0.0);
     }
     // top-k over the lanes (lane e holds expert e), exact ties to the lower id
     int kt = k_per_token ? k_per_token[t] : k;
@@ -523,36 +469,10 @@ __global__ void __launch_bounds__(256) route_block_kernel(
       if (lane == 0) report(status, kStatusDeviceCheck, kWhereRoute, t);
       kt = max(1, min(kt, kcap));
     }
-    bool taken = lane >= E;
-    float sel_v = 0.f;
-    int sel_e = -1;
-    for (int j = 0; j < kt; ++j) {
-      float bv = taken ? -INFINITY : logit;
-      int be = taken ? 0x7FFFFFFF : lane;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if (be == lane) taken = true;
-      if (lane == j) {
-        sel_v = bv;
-        sel_e = be;
-      }
-    }
-    const float lmax = __shfl_sync(0xffffffffu, sel_v, 0);
-    const float z = lane < kt ? expf(sel_v - lmax) : 0.f;
-    float zs = z;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
-    if (lane < k_max) {
-      ids[(size_t)t * k_max + lane] = lane < kt ? sel_e : -1;
-      wout[(size_t)t * k_max + lane] = lane < kt ? z / zs : 0.f;
-    }
+    double sv;
+    int se;
+    warp_select_desc(E, kt, [&](int) { return logit; }, [](int c) { return c; }, sv, se);
+    warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
   }
   if (!do_quant) return;
   float am = red[0];
@@ -598,29 +518,55 @@ cudaError_t launch_route_fused(const Plan& p, const uint16_t* hidden, const floa
   return cudaGetLastError();
 }
 
-cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
-                              const float* bias, int k, const int32_t* k_per_token, float* logits,
-                              int32_t* ids, float* w, uint8_t* xq, float* xs, bool do_quant,
-                              int* status, cudaStream_t s) {
-  const dim3 grid((p.E + 7) / 8);
-  const int q = do_quant ? 1 : 0;
-  if (p.T <= 1)
-    launch_pdl(route_gemv_kernel<1>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
-               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
-  else if (p.T <= 2)
-    launch_pdl(route_gemv_kernel<2>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
-               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
-  else if (p.T <= 4)
-    launch_pdl(route_gemv_kernel<4>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
-               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
-  else
-    launch_pdl(route_gemv_kernel<8>, grid, dim3(256), 0, s, hidden, router_w, bias, p.T, p.d, p.E,
-               k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
+// Sets a kernel's dynamic shared-memory limit once per device (the first launch there).
+template <typename K>
+static cudaError_t allow_dynamic_smem(K kernel, int bytes, bool (&done)[64]) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (err != cudaSuccess) return err;
+    done[dev] = true;
+  }
+  return cudaSuccess;
+}
+
+template <int TT>
+static cudaError_t launch_gemv_t(const Plan& p, const uint16_t* hidden, const float* router_w,
+                                 const float* bias, int k, const int32_t* k_per_token,
+                                 double* logits, int32_t* ids, float* w, uint8_t* xq, float* xs,
+                                 int q, int* status, cudaStream_t s) {
+  static bool done[64] = {};
+  cudaError_t err = allow_dynamic_smem(route_gemv_kernel<TT>, kGemvMaxT * kMaxExperts * 8, done);
+  if (err != cudaSuccess) return err;
+  const size_t smem = sizeof(double) * (size_t)p.T * p.E;
+  launch_pdl(route_gemv_kernel<TT>, dim3((p.E + 7) / 8), dim3(256), smem, s, hidden, router_w,
+             bias, p.T, p.d, p.E, k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
   return cudaGetLastError();
 }
 
+cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
+                              const float* bias, int k, const int32_t* k_per_token,
+                              double* logits, int32_t* ids, float* w, uint8_t* xq, float* xs,
+                              bool do_quant, int* status, cudaStream_t s) {
+  const int q = do_quant ? 1 : 0;
+  if (p.T <= 1)
+    return launch_gemv_t<1>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
+                            status, s);
+  if (p.T <= 2)
+    return launch_gemv_t<2>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
+                            status, s);
+  if (p.T <= 4)
+    return launch_gemv_t<4>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
+                            status, s);
+  return launch_gemv_t<8>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
+                          status, s);
+}
+
 cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
-                                 float* part, cudaStream_t s) {
+                                 double* part, cudaStream_t s) {
   dim3 grid((p.T + kRouterTile - 1) / kRouterTile, (p.E + kRouterTile - 1) / kRouterTile,
             p.r_splits);
   launch_pdl(router_logits_kernel, dim3(grid), dim3(256), 0, s, hidden, router_w, p.T, p.d, p.E,
@@ -628,7 +574,7 @@ cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const fl
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk_quant(const Plan& p, const float* part, const float* bias, int k,
+cudaError_t launch_topk_quant(const Plan& p, const double* part, const float* bias, int k,
                               const int32_t* k_per_token, int32_t* ids, float* w,
                               const uint16_t* hidden, uint8_t* xq, float* xs, bool do_route,
                               bool do_quant, const float* refine_w, int* status, cudaStream_t s) {

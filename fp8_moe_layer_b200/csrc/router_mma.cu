@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
 
 __global__ void __launch_bounds__(256, 1)
     router_mma_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
-                      int T, int E, int num_kb, float* __restrict__ logits, int* status) {
+                      int T, int E, int num_kb, double* __restrict__ logits, int* status) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   extern __shared__ uint8_t smem_raw[];
@@ -202,7 +202,8 @@ __global__ void __launch_bounds__(256, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 16; ++c)
-          if (c0 + c < nvalid && e < E) logits[(size_t)(t0 + c0 + c) * E + e] = __uint_as_float(r[c]);
+          if (c0 + c < nvalid && e < E)
+            logits[(size_t)(t0 + c0 + c) * E + e] = static_cast<double>(__uint_as_float(r[c]));
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
-                              const CUtensorMap& map_w, const CUtensorMap& map_x, float* logits,
+                              const CUtensorMap& map_w, const CUtensorMap& map_x, double* logits,
                               int* status, cudaStream_t s) {
   const int64_t n = (int64_t)p.E * p.d;
   const int split_blocks = (int)std::min<int64_t>((n + 255) / 256, 4LL * num_sms());

@@ -67,6 +67,7 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_forward": (ctypes.c_int, [dims_p, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp,
                                        vp, vp, vp, sz, vp, ctypes.POINTER(MoEDebugOut)]),
         "moe_route_topk_noalloc": (ctypes.c_int, [dims_p, vp, vp, vp, i32, vp, vp, vp, vp]),
+        "moe_kernel_launch_count": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -76,6 +77,16 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 LIB = _load()
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Another build of the same C ABI (e.g. the wait-test build), with the argument types set."""
+    return _load(path)
+
+
+def kernel_launch_count() -> int:
+    """Kernels the library has launched in this process so far (a host-side counter)."""
+    return int(LIB.moe_kernel_launch_count())
 
 
 def status_string(status: int) -> str:
@@ -213,8 +224,9 @@ def moe_combine(expert_out, topk_w, inv_row, shared_out=None, want_f32=False):
 
 def moe_forward(hidden, router_w, router_bias, k, k_per_token, w13, w13_scale, w2, w2_scale,
                 k_max, shared: Optional[Sequence[torch.Tensor]] = None, ws=None, y=None,
-                debug: bool = False, stage_events: Optional[Sequence] = None):
-    """The whole layer. Returns y bf16 [T, d], or (y, dict of debug outputs) when debug=True."""
+                debug: bool = False, stage_events: Optional[Sequence] = None, lib=None):
+    """The whole layer. Returns y bf16 [T, d], or (y, dict of debug outputs) when debug=True.
+    ``lib``: another build of the library loaded with ``load_library`` (default: this one)."""
     T, d = hidden.shape
     E, twoF, _ = w13.shape
     F = twoF // 2
@@ -246,7 +258,7 @@ def moe_forward(hidden, router_w, router_bias, k, k_per_token, w13, w13_scale, w
                                     "inv_row", "y_f32")),
                                  ctypes.cast(ev_arr, ctypes.POINTER(ctypes.c_void_p))
                                  if ev_arr is not None else None)
-    status = LIB.moe_forward(
+    status = (lib or LIB).moe_forward(
         ctypes.byref(dm), _p(_bits(hidden)), _p(router_w), _p(router_bias), int(k),
         _p(k_per_token), _p(_u8(w13)), _p(w13_scale), _p(_u8(w2)), _p(w2_scale), _p(_u8(w13s)),
         _p(s13s), _p(_u8(w2s)), _p(s2s), _p(y.view(torch.int16)), _p(ws), ws.numel(),

@@ -91,6 +91,11 @@ size_t moe_workspace_bytes(const moe_dims* dims);
 /* Host only, pure. A static English description of a moe_status value. */
 const char* moe_status_string(int status);
 
+/* Host only. The number of kernels this library has launched in this process so far (every
+ * device, every host thread), for benchmarks and profiling: its difference across a region of
+ * calls counts the library's launches in that region. Reads a relaxed atomic counter. */
+uint64_t moe_kernel_launch_count(void);
+
 /* Clears the device status word kept at the start of `ws` (16 bytes: error code, where-code,
  * detail, and the completion counter of the one-kernel decode router), async on `stream`.
  * moe_forward clears it itself; callers of the split entry points clear it once after
@@ -101,9 +106,12 @@ int moe_clear_status(void* ws, void* stream);
  * Synchronises `stream`. Returns MOE_ERR_CUDA if the copy or the synchronisation fails. */
 int moe_device_status(const void* ws, void* stream, int32_t* out_status);
 
-/* Router: logits l[t,e] = sum_d hidden[t,d] * router_w[e,d] (+ router_bias[e]) in fp32, softmax
- * over the E experts, the k_t largest (descending; exact ties to the lower expert id) and their
- * probabilities renormalised to sum to 1 ("Routage MoE entre GPU", router paragraph).
+/* Router: logits l[t,e] = sum_d hidden[t,d] * router_w[e,d] (+ router_bias[e]), softmax over the
+ * E experts, the k_t largest (descending; exact ties to the lower expert id) and their
+ * probabilities renormalised to sum to 1 ("Routage MoE entre GPU", router paragraph). The logits
+ * that decide the selection are summed in fp64 (each bf16 x fp32 product is exact there), so the
+ * ids and their order are those of an fp64 evaluation unless two logits lie within ~1e-12; the
+ * weights are computed in fp64 and rounded once to fp32.
  *   hidden [T, d] bf16; router_w [E, d] fp32; router_bias [E] fp32 or NULL;
  *   k: experts per token when k_per_token is NULL (1 <= k <= min(E, k_max));
  *   k_per_token [T] int32 or NULL: per-token k_t in [1, k_max] (MoE-Prism's elastic k);
@@ -171,8 +179,8 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
  * point; it returns the same routing decision as moe_route_topk (same arguments, minus the
  * workspace), computed with the CUDA-core router.
  *   Scratch: one fixed device array of MOE_NOALLOC_SCRATCH_BYTES owned by this library, which
- *   every GPU that loads the library keeps until the process exits. It holds the partial router
- *   logits, 4 * T * E * splits bytes (splits = the number of pieces d is cut into so that the
+ *   every GPU that loads the library keeps until the process exits. It holds the fp64 partial
+ *   router logits, 8 * T * E * splits bytes (splits = the number of pieces d is cut into so that the
  *   logits kernel fills the GPU; none at all for E <= 32); a larger shape returns
  *   MOE_ERR_UNSUPPORTED and launches nothing.
  *   The first call on a device looks up the array's device address (with that device current);

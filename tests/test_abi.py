@@ -80,3 +80,76 @@ def test_host_validation_without_gpu(ops):
     zero = ops.dims(0, 128, 8, 256, 2)
     assert L.moe_forward(ctypes.byref(zero), *([None] * 3), 2, *([None] * 11), 0, None,
                          None) == ops.MOE_OK
+
+
+# The final C signatures, written out: a C file assigns every entry point to a pointer of exactly
+# this type, and gcc rejects any difference (-Werror). The Python binding's argument counts must
+# match too. (Departures from the boundary first sketched are listed in the design notes.)
+SIGNATURES = {
+    "moe_workspace_bytes": "size_t (*)(const moe_dims*)",
+    "moe_status_string": "const char* (*)(int)",
+    "moe_kernel_launch_count": "uint64_t (*)(void)",
+    "moe_clear_status": "int (*)(void*, void*)",
+    "moe_device_status": "int (*)(const void*, void*, int32_t*)",
+    "moe_route_topk": "int (*)(const moe_dims*, const uint16_t*, const float*, const float*, "
+                      "int32_t, const int32_t*, int32_t*, float*, void*, size_t, void*)",
+    "moe_permute": "int (*)(const moe_dims*, const int32_t*, int32_t, const int32_t*, int32_t*, "
+                   "int32_t*, int32_t*, void*, size_t, void*)",
+    "moe_grouped_ffn_fp8": "int (*)(const moe_dims*, const uint16_t*, const uint8_t*, "
+                           "const float*, const uint8_t*, const float*, const int32_t*, "
+                           "const int32_t*, float*, float*, void*, size_t, void*)",
+    "moe_combine": "int (*)(const moe_dims*, const float*, const float*, const int32_t*, "
+                   "const float*, uint16_t*, float*, void*)",
+    "moe_forward": "int (*)(const moe_dims*, const uint16_t*, const float*, const float*, int32_t, "
+                   "const int32_t*, const uint8_t*, const float*, const uint8_t*, const float*, "
+                   "const uint8_t*, const float*, const uint8_t*, const float*, uint16_t*, void*, "
+                   "size_t, void*, const moe_debug_out*)",
+    "moe_route_topk_noalloc": "int (*)(const moe_dims*, const uint16_t*, const float*, "
+                              "const float*, int32_t, const int32_t*, int32_t*, float*, void*)",
+}
+
+
+def _nargs(sig: str) -> int:
+    inner = sig.split("(*)(", 1)[1].rsplit(")", 1)[0].strip()
+    return 0 if inner == "void" else inner.count(",") + 1
+
+
+def test_header_signatures_are_the_final_ones(tmp_path):
+    import shutil
+    import subprocess
+    assert sorted(SIGNATURES) == declared_functions()
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    lines = ['#include "moe.h"']
+    for i, (name, sig) in enumerate(SIGNATURES.items()):
+        ptr = sig.replace("(*)", f"(*p{i})", 1)
+        lines.append(f"{ptr} = {name};")
+    src = tmp_path / "sig.c"
+    src.write_text("\n".join(lines) + "\n")
+    res = subprocess.run([gcc, "-std=c11", "-Wall", "-Werror", "-c", str(src), "-o",
+                          str(tmp_path / "sig.o"), f"-I{os.path.dirname(HEADER)}"],
+                         capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+
+
+def test_binding_argument_counts_match_the_header(ops):
+    for name, sig in SIGNATURES.items():
+        fn = getattr(ops.LIB, name)
+        assert len(fn.argtypes) == _nargs(sig), name
+
+
+def test_wait_test_build_exports_its_switch_and_the_library_does_not():
+    from fp8_moe_layer_b200 import build
+    path = build.build(lib=build.LIB_WAITTEST)
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "moe_testing.h")).read(),
+                  flags=re.S)
+    names = sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+    assert names == ["moe_test_withhold_gemm_commit"]
+    test_lib = ctypes.CDLL(path)
+    prod = ctypes.CDLL(os.path.join(ROOT, "fp8_moe_layer_b200", "libfp8moe.so"))
+    for n in names:
+        assert hasattr(test_lib, n)
+        assert not hasattr(prod, n)
+    for n in declared_functions():
+        assert hasattr(test_lib, n), n

@@ -19,6 +19,10 @@ def ops():
 
 
 def forward_and_check(ops, inp, sample=None, seed=0):
+    """moe_forward through the C ABI against the oracle. Routing and grouping are checked on
+    every token (bit-exact). Outputs: every token, or -- when ``sample`` is given -- the tokens of
+    every active expert's first and last routed rows (so every group's first tile and ragged tail
+    tile is compared) plus ``sample`` tokens at random."""
     s = inp.shape
     d = H.to_cuda(inp)
     dm = ops.dims(s.T, s.d, s.E, s.F, s.k_max, s.F_shared)
@@ -30,25 +34,29 @@ def forward_and_check(ops, inp, sample=None, seed=0):
     gpu = {k: H.np_(v) for k, v in dbg.items()}
 
     # routing on every token, grouping bit-exact against the oracle's sort of the GPU's own ids
+    # (and against the oracle's own grouping when the ids are identical)
     x = O.bf16_bits_to_f64(H.hidden_bits(inp.hidden))
     logits = O.router_logits(x, H.np_(inp.router_w), H.np_(inp.router_bias))
     k_t = O.token_k(s.T, s.k, H.np_(inp.k_per_token))
     ids = O.select_topk(logits, k_t, s.k_max)
     route_ref = dict(logits=logits, topk_ids=ids, topk_w=O.routing_weights(logits, ids), k_t=k_t)
-    n_near, differed, n_order = H.check_routing(gpu["topk_ids"], gpu["topk_w"], route_ref, s.d)
-    H.check_grouping(gpu["expert_offsets"], gpu["perm_token"], gpu["inv_row"],
-                     gpu["topk_ids"], k_t, s.E)
+    n_near, differed, n_exact = H.check_routing(gpu["topk_ids"], gpu["topk_w"], route_ref)
+    same_grouping = H.check_grouping(gpu["expert_offsets"], gpu["perm_token"], gpu["inv_row"],
+                                     gpu["topk_ids"], k_t, s.E, ref_ids=ids)
 
-    # outputs: all tokens, or a sample of tokens without a near tie
-    near = set(O.near_tie_tokens(logits, k_t, H.NEAR_TIE).tolist())
-    tokens = np.array([t for t in range(s.T) if t not in near], dtype=np.int64)
-    if sample is not None and len(tokens) > sample:
-        rng = np.random.default_rng(seed)
-        tokens = np.sort(rng.choice(tokens, size=sample, replace=False))
+    # outputs: every token whose routing equals the oracle's (all but exact fp64 ties)
+    agree = np.all(gpu["topk_ids"] == ids, axis=1)
+    if sample is None:
+        tokens = np.arange(s.T)
+    else:
+        tokens = H.coverage_tokens(gpu["expert_offsets"], gpu["perm_token"], s.E, s.T, sample,
+                                   seed=seed, shared=bool(s.F_shared))
+    tokens = tokens[agree[tokens]]
     ref = H.run_oracle(inp, tokens=tokens)
     stats = H.check_output(y[tokens], torch.from_numpy(gpu["y_f32"][tokens]), ref["y64"], s.name)
-    print(f"{s.name}: tokens checked {len(tokens)}/{s.T}, near ties {n_near} "
-          f"(differing {differed}), order-only ties {n_order}, {stats}")
+    print(f"{s.name}: tokens checked {len(tokens)}/{s.T}, near ties (<{H.NEAR_TIE:g}) {n_near} "
+          f"(differing {differed}), exact ties (<{H.EXACT_TIE:g}) {n_exact}, grouping equal to "
+          f"the oracle's {same_grouping}, {stats}")
     return y, dbg, stats
 
 
@@ -110,9 +118,10 @@ def test_forward_is_deterministic(ops):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
-FULL = [("mixtral_T1", None), ("mixtral_T32", 12), ("mixtral_T512", 12), ("qwen3_T1", None),
-        ("qwen3_T64", None), ("qwen3_T4096", 16), ("prism_T64", None), ("prism_T2048", 16),
-        ("deepseek_T128", 8)]
+# (workload, random tokens beside every expert's first- and last-row tokens; None = every token)
+FULL = [("mixtral_T1", None), ("mixtral_T32", None), ("mixtral_T512", 128), ("qwen3_T1", None),
+        ("qwen3_T64", None), ("qwen3_T4096", 128), ("prism_T64", None), ("prism_T2048", 128),
+        ("deepseek_T128", None)]
 
 
 @pytest.mark.parametrize("name,sample", FULL, ids=[f[0] for f in FULL])
@@ -121,4 +130,4 @@ def test_forward_full_size_workloads(ops, name, sample):
 
 
 def test_forward_deepseek_prefill(ops):
-    forward_and_check(ops, H.make_inputs(I.WORKLOADS["deepseek_T8192"], seed=0), sample=8)
+    forward_and_check(ops, H.make_inputs(I.WORKLOADS["deepseek_T8192"], seed=0), sample=64)

@@ -1,6 +1,6 @@
-"""CUDA-graph executor of the layer (one graph per token bucket and k profile): a replay equals
-the eager moe_forward of the padded batch bit for bit, and matches the unpadded eager call on
-the real tokens within the output tolerance; inputs change between replays."""
+"""CUDA-graph executor of the layer (one graph per token bucket and k profile): a replay matches
+the oracle on the real tokens within the output tolerance, equals the eager moe_forward of the
+padded batch bit for bit, and matches the unpadded eager call; inputs change between replays."""
 import numpy as np
 import pytest
 import torch
@@ -40,6 +40,9 @@ def test_graph_replay_matches_eager(ops, shape, T):
         y_graph = ex(h, kpt).clone()
         torch.cuda.synchronize()
         assert ex.device_status() == ops.MOE_OK
+        # the oracle on the same real tokens
+        ref = H.run_oracle_on(inp, h, kpt)
+        H.check_output(y_graph, None, ref["y64"], f"{shape.name} graph replay {rep}")
         # the same padded batch through the eager call: identical bits
         hp = _pad(h, T_b)
         kp = None

@@ -1,5 +1,6 @@
-"""k-aware batching on the GPU: the tiered fixed-k calls (eager and graph-replayed) give every
-token the output of the one-call elastic layer, within the output tolerance."""
+"""k-aware batching on the GPU: the tiered fixed-k calls (eager and graph-replayed) match the
+oracle on every token, and the output of the one-call elastic layer, within the output
+tolerance."""
 import pytest
 import torch
 
@@ -29,3 +30,5 @@ def test_tiered_equals_elastic(shape, graphs):
     assert ops.device_status(layer.ws) == ops.MOE_OK
     diff = (y_t - y_e).abs().max().item()
     assert diff <= H.Y_ATOL + 0.5 ** 8 * y_e.abs().max().item(), diff
+    ref = H.run_oracle(inp)
+    H.check_output(y_t.to(torch.bfloat16), None, ref["y64"], f"{shape.name} tiered")

@@ -58,9 +58,9 @@ def test_route_topk_matches_oracle(ops, shape):
     ref = _oracle_route(shape, hidden, rw, rb, kpt)
     c = lambda t: None if t is None else t.cuda()
     ids, w = ops.moe_route_topk(c(hidden), c(rw), c(rb), shape.k, c(kpt), shape.k_max)
-    n_near, differed, n_order = H.check_routing(H.np_(ids), H.np_(w), ref, shape.d)
-    print(f"{shape.name}: near-tie tokens {n_near}, differing among them {differed}, "
-          f"order-only ties {n_order}")
+    n_near, differed, n_exact = H.check_routing(H.np_(ids), H.np_(w), ref)
+    print(f"{shape.name}: near-tie tokens (<{H.NEAR_TIE:g}) {n_near}, differing among them "
+          f"{differed}, exact ties (<{H.EXACT_TIE:g}) {n_exact}")
 
 
 def _random_ids(T, E, k_max, k_t, rng, skew=None):
