@@ -29,7 +29,7 @@ struct Plan {
   int g1_splits, g1_kb_per_split;             // gate/up K split (decode); 1 = SwiGLU epilogue
   int g2_kb, g2_m_tiles, g2_splits, g2_kb_per_split;  // down GEMM
   size_t off_status, off_part, off_ids, off_w, off_offsets, off_tiles, off_perm, off_inv, off_pscr;
-  size_t off_xq, off_xs, off_xqp, off_xsp, off_amax, off_act, off_aq, off_s2, off_o, off_planes;
+  size_t off_xq, off_xs, off_amax, off_act, off_aq, off_s2, off_o, off_planes;
   size_t off_hpart;
   size_t bytes;
 };
@@ -47,7 +47,12 @@ struct GemmArgs {
   int G, E_routed;               // groups >= E_routed use the shared-expert weights
   int m_tiles, splits, kb_per_split, num_kb;
   int M_valid;                   // valid weight rows: F (gate/up halves) or d (down)
-  const float* row_scale;        // [Rpad] activation scale of each routed row
+  const float* row_scale;        // down: [Rpad] activation scale of each routed row
+  // gate/up: token rows fetched through the permutation (tile::gather4 loads from the quantised
+  // hidden states [T, d]); scale of routed row r = token_scale[row_token[r]]
+  const int32_t* row_token;      // [Rpad] token of each routed row
+  const float* token_scale;      // [T]
+  int T;
   const float* w_scale;          // [E, w_scale_ld] per-output-channel weight scales
   const float* w_scale_shared;   // [w_scale_ld] shared expert (or null)
   int w_scale_ld;                // 2F (gate/up) or d (down)
@@ -82,7 +87,8 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est 
 // Router logits are fp64 (part [splits][T][E] doubles): see route.cu.
 cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
                                  double* part, cudaStream_t s);
-cudaError_t launch_topk_quant(const Plan& p, const double* part, const float* bias, int k,
+// With refine_w (the tensor-core path) `part` also serves as scratch for rare tokens.
+cudaError_t launch_topk_quant(const Plan& p, double* part, const float* bias, int k,
                               const int32_t* k_per_token, int32_t* ids, float* w,
                               const uint16_t* hidden, uint8_t* xq, float* xs, bool do_route,
                               bool do_quant, const float* refine_w, int* status, cudaStream_t s);
@@ -120,22 +126,14 @@ cudaError_t launch_route_fused(const Plan& p, const uint16_t* hidden, const floa
                                int* status, cudaStream_t s);
 // scratch: 2 * permute_blocks(p) * E int32 (per-block counts and bases; unused for one block)
 int permute_blocks(const Plan& p);
-// grouping + row gather in one kernel (when the grouping fits one block, T * k_max <= 8192)
-bool permute_gather_fused(const Plan& p);
-cudaError_t launch_permute_gather(const Plan& p, const int32_t* ids, int k,
-                                  const int32_t* k_per_token, int32_t* offsets, int32_t* perm,
-                                  int32_t* inv, int32_t* tiles, const uint8_t* xq, const float* xs,
-                                  uint8_t* xqp, float* xsp, uint32_t* amax, int* status,
-                                  cudaStream_t s);
+// Grouping; also zeroes amax[r] of every routed (and shared) row when amax is given.
 cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
-                           int32_t* scratch, int* status, cudaStream_t s);
+                           int32_t* scratch, uint32_t* amax, int* status, cudaStream_t s);
 cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* tiles, int* status,
                                cudaStream_t s);
-cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, const int32_t* perm,
-                          const int32_t* total_rows, uint8_t* xqp, float* xsp, uint32_t* amax,
-                          int* status, cudaStream_t s);
-// acts64 / acts16: the routed-row activations with 64-row and 16-row TMA boxes
+// gate/up: acts64 = the quantised hidden states with one-row boxes (gather4; acts16 unused);
+// down: acts64 / acts16 = the routed-row activations with 64-row and 16-row TMA boxes
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
                                const CUtensorMap& acts64, const CUtensorMap& acts16,
                                const GemmArgs& a, bool partial, cudaStream_t s);

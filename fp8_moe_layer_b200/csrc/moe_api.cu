@@ -99,10 +99,11 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
 #ifdef MOE_FORCE_PAIR
   p->pair1 = p->pair2 = MOE_FORCE_PAIR;
 #endif
-  // A prefill gate/up CTA holds two 128-row weight slabs against one token tile (two TMEM
-  // accumulators): the token rows cross L2 -> shared memory once per 512 weight rows of a pair,
-  // a quarter fewer bytes per MMA than one slab.
-  p->slabs1 = p->pair1 ? 2 : 1;
+  // Weight slabs per gate/up CTA. Two slabs (two TMEM accumulators against one token tile: a
+  // quarter fewer L2 -> shared-memory bytes per MMA) measured slower on B200 than one -- DeepSeek
+  // T=8192 gate/up 2802 vs 2659 us, Mixtral T=512 layer 352 vs 317 us: only four pipeline stages
+  // fit, and tiles wider than 128 tokens lose the accumulator double buffering -- so one.
+  p->slabs1 = 1;
 #ifdef MOE_FORCE_SLABS
   p->slabs1 = p->pair1 ? MOE_FORCE_SLABS : 1;
 #endif
@@ -153,8 +154,6 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   p->off_pscr = take(sizeof(int32_t) * 2 * (size_t)permute_blocks(*p) * E);
   p->off_xq = take((size_t)T * d);
   p->off_xs = take(sizeof(float) * (size_t)T);
-  p->off_xqp = take((size_t)p->Rpad * d);
-  p->off_xsp = take(sizeof(float) * (size_t)p->Rpad);
   p->off_amax = take(sizeof(uint32_t) * (size_t)p->Rpad);
   p->off_act = take(sizeof(float) * (size_t)p->Rpad * F);
   p->off_aq = take((size_t)p->Rpad * F);
@@ -245,6 +244,13 @@ static bool map_w2(CUtensorMap* m, const uint8_t* w, int experts, int d, int F) 
   const uint32_t box[3] = {(uint32_t)kBK, 128, 1};
   return make_map(m, w, 3, dims, str, box);
 }
+// Quantised hidden states [T, d] for tile::gather4 loads: box 128 (K) x 1 row.
+static bool map_token_rows(CUtensorMap* m, const uint8_t* xq, int T, int d) {
+  const uint64_t dims[2] = {(uint64_t)d, (uint64_t)std::max(T, 1)};
+  const uint64_t str[1] = {(uint64_t)d};
+  const uint32_t box[2] = {(uint32_t)kBK, 1};
+  return make_map(m, xq, 2, dims, str, box);
+}
 // Row-major activations [rows, K]: box 128 (K) x BN rows.
 static bool map_rows(CUtensorMap* m, const uint8_t* a, int64_t rows, int K, int BN) {
   const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
@@ -272,10 +278,10 @@ static int check_device() {
 struct Ws {
   int* status;
   double* part;
-  float *w, *xs, *xsp, *act, *s2, *o, *hpart;
+  float *w, *xs, *act, *s2, *o, *hpart;
   uint16_t* planes;
   int32_t *ids, *offsets, *tiles, *perm, *inv, *pscr;
-  uint8_t *xq, *xqp, *aq;
+  uint8_t *xq, *aq;
   uint32_t* amax;
 };
 
@@ -293,8 +299,6 @@ static Ws carve(const Plan& p, void* ws) {
   w.pscr = reinterpret_cast<int32_t*>(b + p.off_pscr);
   w.xq = b + p.off_xq;
   w.xs = reinterpret_cast<float*>(b + p.off_xs);
-  w.xqp = b + p.off_xqp;
-  w.xsp = reinterpret_cast<float*>(b + p.off_xsp);
   w.amax = reinterpret_cast<uint32_t*>(b + p.off_amax);
   w.act = reinterpret_cast<float*>(b + p.off_act);
   w.aq = b + p.off_aq;
@@ -345,10 +349,10 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
                    const uint8_t* w2, const float* w2_scale, const uint8_t* w13s,
                    const float* w13s_scale, const uint8_t* w2s, const float* w2s_scale,
                    float* o, size_t split_stride, int64_t o_rows, void* const* ev,
-                   cudaStream_t s, bool gathered = false) {
-  CUtensorMap m13, m13s, mxq64, mxq16, m2, m2s, maq64, maq16;
+                   cudaStream_t s) {
+  CUtensorMap m13, m13s, mxq, m2, m2s, maq64, maq16;
   if (!map_w13(&m13, w13, p.E, p.F, p.d) || !map_w2(&m2, w2, p.E, p.d, p.F) ||
-      !map_rows(&mxq64, w.xqp, p.Rpad, p.d, 64) || !map_rows(&mxq16, w.xqp, p.Rpad, p.d, 16) ||
+      !map_token_rows(&mxq, w.xq, p.T, p.d) ||
       !map_rows(&maq64, w.aq, p.Rpad, p.F, 64) || !map_rows(&maq16, w.aq, p.Rpad, p.F, 16))
     return MOE_ERR_UNSUPPORTED;
   m13s = m13;
@@ -362,9 +366,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   };
   const int32_t* total_rows = w.offsets + p.G;     // offsets[G] = routed (+ shared) rows
 
-  record(3);
-  if (!gathered)   // (else the grouping kernel already laid the rows out)
-    MOE_CUDA(launch_gather(p, w.xq, w.xs, w.perm, total_rows, w.xqp, w.xsp, w.amax, w.status, s));
+  record(3);      // (no row gather: the gate/up GEMM fetches token rows through the permutation)
 
   GemmArgs g1{};
   g1.group_offsets = w.offsets;
@@ -376,7 +378,10 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g1.kb_per_split = p.g1_kb;
   g1.num_kb = p.g1_kb;
   g1.M_valid = p.F;
-  g1.row_scale = w.xsp;
+  g1.row_scale = nullptr;
+  g1.row_token = w.perm;
+  g1.token_scale = w.xs;
+  g1.T = p.T;
   g1.w_scale = w13_scale;
   g1.w_scale_shared = w13s_scale;
   g1.w_scale_ld = 2 * p.F;
@@ -398,7 +403,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
     g1.row_amax = nullptr;
   }
   record(4);
-  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mxq64, mxq16, g1, split1, s));
+  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mxq, mxq, g1, split1, s));
 
   record(5);
   if (split1)
@@ -414,6 +419,8 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g2.num_kb = p.g2_kb;
   g2.M_valid = p.d;
   g2.row_scale = w.s2;
+  g2.row_token = nullptr;
+  g2.token_scale = nullptr;
   g2.w_scale = w2_scale;
   g2.w_scale_shared = w2s_scale;
   g2.w_scale_ld = p.d;
@@ -540,7 +547,7 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_ids, int32_t k,
   q.shared = false;
   q.G = p.E;
   MOE_CUDA(launch_permute(q, topk_ids, k, k_per_token, expert_offsets, perm_token, inv_row,
-                          w.tiles, w.pscr, w.status, static_cast<cudaStream_t>(stream)));
+                          w.tiles, w.pscr, nullptr, w.status, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
@@ -575,6 +582,7 @@ int moe_grouped_ffn_fp8(const moe_dims* dims, const uint16_t* hidden, const uint
   MOE_CUDA(cudaMemcpyAsync(w.offsets, expert_offsets, sizeof(int32_t) * (p.E + 1),
                            cudaMemcpyDeviceToDevice, s));
   MOE_CUDA(cudaMemcpyAsync(w.perm, perm_token, sizeof(int32_t) * q.Rcap, cudaMemcpyDeviceToDevice, s));
+  MOE_CUDA(cudaMemsetAsync(w.amax, 0, sizeof(uint32_t) * q.Rcap, s));   // the requant's row maxima
   const bool direct = p.g2_splits == 1;
   MOE_TRY(run_ffn(q, w, w13, w13_scale, w2, w2_scale, nullptr, nullptr, nullptr, nullptr,
                   direct ? expert_out : w.o, (size_t)p.Rpad * p.d, q.Rcap, nullptr, s));
@@ -651,16 +659,11 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                                w.status, s));
   }
   record(2);
-  const bool fused = permute_gather_fused(p);
-  if (fused)
-    MOE_CUDA(launch_permute_gather(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles,
-                                   w.xq, w.xs, w.xqp, w.xsp, w.amax, w.status, s));
-  else
-    MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
-                            w.status, s));
+  MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
+                          w.amax, w.status, s));
   const size_t split_stride = (size_t)p.Rpad * p.d;
   MOE_TRY(run_ffn(p, w, w13, w13_scale, w2, w2_scale, w13_shared, w13s_scale, w2_shared,
-                  w2s_scale, w.o, split_stride, p.Rcap, ev, s, fused));
+                  w2s_scale, w.o, split_stride, p.Rcap, ev, s));
   record(7);
   MOE_CUDA(launch_combine(p, w.o, p.g2_splits, split_stride, w.w, w.inv,
                           p.shared ? w.o : nullptr, p.shared ? w.offsets + p.E : nullptr,

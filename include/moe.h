@@ -71,9 +71,9 @@ typedef struct moe_dims {
  *     event i is recorded on `stream` just before stage i's kernel, the last one after the last
  *     stage. Stages: 0 router logits, 1 top-k + activation quantisation, 2 permutation,
  *     3 row gather, 4 gate/up GEMM + SwiGLU, 5 intermediate requantisation, 6 down GEMM,
- *     7 combine. A stage computed by the previous stage's kernel brackets nothing: stage 1 when
- *     one kernel routes and quantises (E <= 32, or decode batches of T <= 8), stage 3 when one
- *     kernel groups and gathers the rows (T * k_max <= 8192). */
+ *     7 combine. A stage computed by another stage's kernel brackets nothing: stage 1 when one
+ *     kernel routes and quantises (E <= 32, or decode batches of T <= 8), and stage 3 always
+ *     (the gate/up GEMM fetches the token rows through the permutation itself). */
 #define MOE_NUM_STAGES 8
 typedef struct moe_debug_out {
   int32_t* topk_ids;
