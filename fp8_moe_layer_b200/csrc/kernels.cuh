@@ -28,9 +28,13 @@ struct Plan {
   int g1_kb, g1_m_tiles;                      // gate/up GEMM: K blocks (d/128), 64-row tiles
   int g1_splits, g1_kb_per_split;             // gate/up K split (decode); 1 = SwiGLU epilogue
   int g2_kb, g2_m_tiles, g2_splits, g2_kb_per_split;  // down GEMM
+  // decode tiles (BN <= 64): the gate/up GEMM always writes K-split partials and applies SwiGLU +
+  // requantisation itself (per token tile); fuse_combine: the down GEMM also combines (T <= 16)
+  bool fuse_swiglu, fuse_combine;
+  int n_tiles_cap;   // bound on the tile prefix: counters of the fused epilogues
   size_t off_status, off_part, off_ids, off_w, off_offsets, off_tiles, off_perm, off_inv, off_pscr;
-  size_t off_xq, off_xs, off_amax, off_act, off_aq, off_s2, off_o, off_planes;
-  size_t off_hpart;
+  size_t off_xq, off_xs, off_xqp, off_xsp, off_amax, off_act, off_aq, off_s2, off_o, off_planes;
+  size_t off_hpart, off_counters;
   size_t bytes;
 };
 
@@ -48,8 +52,9 @@ struct GemmArgs {
   int m_tiles, splits, kb_per_split, num_kb;
   int M_valid;                   // valid weight rows: F (gate/up halves) or d (down)
   const float* row_scale;        // down: [Rpad] activation scale of each routed row
-  // gate/up: token rows fetched through the permutation (tile::gather4 loads from the quantised
-  // hidden states [T, d]); scale of routed row r = token_scale[row_token[r]]
+  // gate/up with decode tiles (BN <= 64): token rows fetched through the permutation
+  // (tile::gather4 loads from the quantised hidden states [T, d]); the scale of routed row r is
+  // token_scale[row_token[r]] instead of row_scale[r]
   const int32_t* row_token;      // [Rpad] token of each routed row
   const float* token_scale;      // [T]
   int T;
@@ -61,6 +66,23 @@ struct GemmArgs {
   size_t out_split_stride;       // elements between split partials
   uint32_t* row_amax;            // gate/up: [Rpad] |act| max as fp32 bits
   int* status;
+  // Decode fusions (null counters = off). K-split gate/up: tile_done[tp[g] + n] counts the
+  // finished tiles of token tile n of group g; the CTA that finishes the last one applies SwiGLU
+  // and the FP8 requantisation to those rows (aq, s2 [Rpad], F = act width). Down: tile_done[m]
+  // counts the finished tiles of output-channel tile m; the CTA that finishes the last one
+  // computes the weighted combine of every token for those channels (y, y_f32 [T, d]; topk_w,
+  // inv_row [T, k_max]; the shared expert's rows follow the routed ones). Each last CTA resets
+  // its counter, so the counters stay zero between calls.
+  int* tile_done;
+  uint8_t* aq;
+  float* s2;
+  int F;
+  const float* topk_w;
+  const int32_t* inv_row;
+  int k_max;
+  int has_shared;
+  uint16_t* y;
+  float* y_f32;
 #ifdef MOE_WAIT_TEST
   int withhold;                  // wait-test build: skip the first tile's accumulator signal
 #endif
@@ -87,8 +109,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est 
 // Router logits are fp64 (part [splits][T][E] doubles): see route.cu.
 cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
                                  double* part, cudaStream_t s);
-// With refine_w (the tensor-core path) `part` also serves as scratch for rare tokens.
-cudaError_t launch_topk_quant(const Plan& p, double* part, const float* bias, int k,
+cudaError_t launch_topk_quant(const Plan& p, const double* part, const float* bias, int k,
                               const int32_t* k_per_token, int32_t* ids, float* w,
                               const uint16_t* hidden, uint8_t* xq, float* xs, bool do_route,
                               bool do_quant, const float* refine_w, int* status, cudaStream_t s);
@@ -112,10 +133,22 @@ inline bool router_uses_gemv(int E, int T, int d) {
   return E > 32 && T >= 1 && T <= 8 && !router_uses_mma(E, T, d);
 }
 inline bool router_uses_gemv(const Plan& p) { return router_uses_gemv(p.E, p.T, p.d); }
+// Grouping done by the decode router's last block (null offsets: routing only). Same outputs as
+// launch_permute (offsets [E+2], perm, inv, tiles [E+2] with the shared expert's group when
+// has_shared), and amax zeroed for every routed / shared row.
+struct DecodeGrouping {
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
+  int32_t* tiles;
+  uint32_t* amax;
+  int BN, has_shared;
+};
 cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
                               const float* bias, int k, const int32_t* k_per_token,
                               double* logits, int32_t* ids, float* w, uint8_t* xq, float* xs,
-                              bool do_quant, int* status, cudaStream_t s);
+                              bool do_quant, int* status, const DecodeGrouping& grp,
+                              cudaStream_t s);
 // planes: 3 * E * d bf16 (workspace); map_w over planes [3][E][d], map_x over hidden [T][d]
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
                               const CUtensorMap& map_w, const CUtensorMap& map_x, double* logits,
@@ -126,14 +159,24 @@ cudaError_t launch_route_fused(const Plan& p, const uint16_t* hidden, const floa
                                int* status, cudaStream_t s);
 // scratch: 2 * permute_blocks(p) * E int32 (per-block counts and bases; unused for one block)
 int permute_blocks(const Plan& p);
-// Grouping; also zeroes amax[r] of every routed (and shared) row when amax is given.
+// grouping + row gather in one kernel (when the grouping fits one block, T * k_max <= 8192)
+bool permute_gather_fused(const Plan& p);
+cudaError_t launch_permute_gather(const Plan& p, const int32_t* ids, int k,
+                                  const int32_t* k_per_token, int32_t* offsets, int32_t* perm,
+                                  int32_t* inv, int32_t* tiles, const uint8_t* xq, const float* xs,
+                                  uint8_t* xqp, float* xsp, uint32_t* amax, int* status,
+                                  cudaStream_t s);
 cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
-                           int32_t* scratch, uint32_t* amax, int* status, cudaStream_t s);
+                           int32_t* scratch, int* status, cudaStream_t s);
 cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* tiles, int* status,
                                cudaStream_t s);
-// gate/up: acts64 = the quantised hidden states with one-row boxes (gather4; acts16 unused);
-// down: acts64 / acts16 = the routed-row activations with 64-row and 16-row TMA boxes
+cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, const int32_t* perm,
+                          const int32_t* total_rows, uint8_t* xqp, float* xsp, uint32_t* amax,
+                          int* status, cudaStream_t s);
+// acts64 / acts16: the B rows' maps -- the routed-row activations with 64-row and 16-row TMA
+// boxes, or (gate/up with decode tiles) the quantised hidden states with one-row boxes for
+// tile::gather4 (acts16 then unused)
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
                                const CUtensorMap& acts64, const CUtensorMap& acts16,
                                const GemmArgs& a, bool partial, cudaStream_t s);

@@ -134,6 +134,10 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
     p->g1_kb_per_split = (int)ceil_div(p->g1_kb, s1);
     p->g1_splits = (int)ceil_div(p->g1_kb, p->g1_kb_per_split);
   }
+  // decode tiles: SwiGLU + requantisation in the gate/up GEMM (one launch less), and for a handful
+  // of tokens the weighted combine in the down GEMM (one more)
+  p->fuse_swiglu = BN <= 64;
+  p->fuse_combine = BN <= 64 && T <= 16;
   const int m_rows2 = p->pair2 ? 256 : 128;      // weight rows of one down-GEMM work unit
   int s2 = choose_splits(est_ntiles * ceil_div(p->g2_m_tiles, m_rows2 / 128), p->g2_kb,
                          p->pair2 ? kPlanSMs / 2 : kPlanSMs, (double)m_rows2 * F,
@@ -143,7 +147,11 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
 
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + std::max<size_t>(bytes, 1)); return o; };
+  p->n_tiles_cap = (int)(ceil_div(p->Rcap, BN) + p->G + 2);
   p->off_status = take(256);
+  // counters of the fused decode epilogues, right after the status word: moe_forward clears both
+  // with one memset
+  p->off_counters = take(sizeof(int) * (size_t)std::max(p->n_tiles_cap, p->g2_m_tiles));
   p->off_part = take(sizeof(double) * (size_t)p->r_splits * T * E);
   p->off_ids = take(sizeof(int32_t) * (size_t)routed);
   p->off_w = take(sizeof(float) * (size_t)routed);
@@ -154,13 +162,17 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   p->off_pscr = take(sizeof(int32_t) * 2 * (size_t)permute_blocks(*p) * E);
   p->off_xq = take((size_t)T * d);
   p->off_xs = take(sizeof(float) * (size_t)T);
+  // permuted copy of the quantised token rows: prefill-sized tiles only (decode tiles gather)
+  p->off_xqp = take(BN >= 128 ? (size_t)p->Rpad * d : 0);
+  p->off_xsp = take(BN >= 128 ? sizeof(float) * (size_t)p->Rpad : 0);
   p->off_amax = take(sizeof(uint32_t) * (size_t)p->Rpad);
   p->off_act = take(sizeof(float) * (size_t)p->Rpad * F);
   p->off_aq = take((size_t)p->Rpad * F);
   p->off_s2 = take(sizeof(float) * (size_t)p->Rpad);
   p->off_o = take(sizeof(float) * (size_t)p->g2_splits * p->Rpad * d);
   p->off_planes = take(router_uses_mma(E, T, d) ? 3 * sizeof(uint16_t) * (size_t)E * d : 0);
-  p->off_hpart = take(p->g1_splits > 1 ? sizeof(float) * p->g1_splits * (size_t)p->Rcap * 2 * F : 0);
+  p->off_hpart = take(p->g1_splits > 1 || p->fuse_swiglu
+                          ? sizeof(float) * p->g1_splits * (size_t)p->Rcap * 2 * F : 0);
   p->bytes = off;
   return MOE_OK;
 }
@@ -278,10 +290,11 @@ static int check_device() {
 struct Ws {
   int* status;
   double* part;
-  float *w, *xs, *act, *s2, *o, *hpart;
+  float *w, *xs, *xsp, *act, *s2, *o, *hpart;
   uint16_t* planes;
   int32_t *ids, *offsets, *tiles, *perm, *inv, *pscr;
-  uint8_t *xq, *aq;
+  int* counters;
+  uint8_t *xq, *xqp, *aq;
   uint32_t* amax;
 };
 
@@ -299,6 +312,8 @@ static Ws carve(const Plan& p, void* ws) {
   w.pscr = reinterpret_cast<int32_t*>(b + p.off_pscr);
   w.xq = b + p.off_xq;
   w.xs = reinterpret_cast<float*>(b + p.off_xs);
+  w.xqp = b + p.off_xqp;
+  w.xsp = reinterpret_cast<float*>(b + p.off_xsp);
   w.amax = reinterpret_cast<uint32_t*>(b + p.off_amax);
   w.act = reinterpret_cast<float*>(b + p.off_act);
   w.aq = b + p.off_aq;
@@ -306,6 +321,7 @@ static Ws carve(const Plan& p, void* ws) {
   w.o = reinterpret_cast<float*>(b + p.off_o);
   w.planes = reinterpret_cast<uint16_t*>(b + p.off_planes);
   w.hpart = reinterpret_cast<float*>(b + p.off_hpart);
+  w.counters = reinterpret_cast<int*>(b + p.off_counters);
   return w;
 }
 
@@ -343,16 +359,34 @@ static int run_router_logits(const Plan& p, const Ws& w, const uint16_t* hidden,
   return MOE_OK;
 }
 
-// Grouped FFN core shared by moe_forward and moe_grouped_ffn_fp8: gather, gate/up GEMM +
-// SwiGLU, requantisation, down GEMM into `o` (split partials `split_stride` apart).
+// Grouped FFN: gate/up GEMM + SwiGLU, requantisation, down GEMM into `o` (split partials
+// `split_stride` apart).
+// Outputs of the weighted combine when the down GEMM computes it (decode fusion).
+struct CombineOut {
+  const float* topk_w;
+  const int32_t* inv_row;
+  uint16_t* y;
+  float* y_f32;
+};
+
+// Grouped FFN core shared by moe_forward and moe_grouped_ffn_fp8. `fuse` (moe_forward only)
+// allows the decode fusions of the plan; returns whether the down GEMM also combined into y.
 static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* w13_scale,
                    const uint8_t* w2, const float* w2_scale, const uint8_t* w13s,
                    const float* w13s_scale, const uint8_t* w2s, const float* w2s_scale,
                    float* o, size_t split_stride, int64_t o_rows, void* const* ev,
-                   cudaStream_t s) {
-  CUtensorMap m13, m13s, mxq, m2, m2s, maq64, maq16;
-  if (!map_w13(&m13, w13, p.E, p.F, p.d) || !map_w2(&m2, w2, p.E, p.d, p.F) ||
-      !map_token_rows(&mxq, w.xq, p.T, p.d) ||
+                   cudaStream_t s, const CombineOut* fuse, bool* combined,
+                   bool gathered = false) {
+  *combined = false;
+  // gate/up B rows: decode tiles fetch token rows through the permutation (gather4), prefill
+  // tiles read the gathered copy
+  const bool gather4 = p.BN <= 64;
+  CUtensorMap m13, m13s, mx64, mx16, m2, m2s, maq64, maq16;
+  const bool maps_x = gather4 ? map_token_rows(&mx64, w.xq, p.T, p.d) &&
+                                    map_token_rows(&mx16, w.xq, p.T, p.d)
+                              : map_rows(&mx64, w.xqp, p.Rpad, p.d, 64) &&
+                                    map_rows(&mx16, w.xqp, p.Rpad, p.d, 16);
+  if (!map_w13(&m13, w13, p.E, p.F, p.d) || !map_w2(&m2, w2, p.E, p.d, p.F) || !maps_x ||
       !map_rows(&maq64, w.aq, p.Rpad, p.F, 64) || !map_rows(&maq16, w.aq, p.Rpad, p.F, 16))
     return MOE_ERR_UNSUPPORTED;
   m13s = m13;
@@ -366,7 +400,9 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   };
   const int32_t* total_rows = w.offsets + p.G;     // offsets[G] = routed (+ shared) rows
 
-  record(3);      // (no row gather: the gate/up GEMM fetches token rows through the permutation)
+  record(3);
+  if (!gather4 && !gathered)   // (else the grouping kernel already laid the rows out)
+    MOE_CUDA(launch_gather(p, w.xq, w.xs, w.perm, total_rows, w.xqp, w.xsp, w.amax, w.status, s));
 
   GemmArgs g1{};
   g1.group_offsets = w.offsets;
@@ -378,7 +414,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g1.kb_per_split = p.g1_kb;
   g1.num_kb = p.g1_kb;
   g1.M_valid = p.F;
-  g1.row_scale = nullptr;
+  g1.row_scale = w.xsp;
   g1.row_token = w.perm;
   g1.token_scale = w.xs;
   g1.T = p.T;
@@ -393,7 +429,8 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
 #ifdef MOE_WAIT_TEST
   g1.withhold = g_withhold_gemm_commit;
 #endif
-  const bool split1 = p.g1_splits > 1;
+  const bool fuse_swiglu = fuse && p.fuse_swiglu;
+  const bool split1 = p.g1_splits > 1 || fuse_swiglu;
   if (split1) {
     g1.splits = p.g1_splits;
     g1.kb_per_split = p.g1_kb_per_split;
@@ -402,15 +439,24 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
     g1.out_split_stride = (size_t)p.Rcap * 2 * p.F;
     g1.row_amax = nullptr;
   }
+  if (fuse_swiglu) {     // SwiGLU + requantisation by the CTA that finishes a token tile
+    g1.tile_done = w.counters;
+    g1.aq = w.aq;
+    g1.s2 = w.s2;
+    g1.F = p.F;
+  }
   record(4);
-  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mxq, mxq, g1, split1, s));
+  MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mx64, mx16, g1, split1, s));
 
   record(5);
-  if (split1)
+  if (fuse_swiglu) {
+    // (computed by the gate/up GEMM)
+  } else if (split1) {
     MOE_CUDA(launch_swiglu_requant(p, w.hpart, p.g1_splits, g1.out_split_stride, total_rows, w.aq,
                                    w.s2, s));
-  else
+  } else {
     MOE_CUDA(launch_requant(p, w.act, w.amax, total_rows, w.aq, w.s2, s));
+  }
 
   GemmArgs g2 = g1;
   g2.m_tiles = p.g2_m_tiles;
@@ -428,9 +474,20 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g2.out_ld = p.d;
   g2.out_split_stride = split_stride;
   g2.row_amax = nullptr;
+  g2.tile_done = nullptr;
 #ifdef MOE_WAIT_TEST
   g2.withhold = 0;
 #endif
+  if (fuse && p.fuse_combine) {   // the weighted combine by the CTA that finishes a channel tile
+    g2.tile_done = w.counters;
+    g2.topk_w = fuse->topk_w;
+    g2.inv_row = fuse->inv_row;
+    g2.k_max = p.k_max;
+    g2.has_shared = p.shared ? 1 : 0;
+    g2.y = fuse->y;
+    g2.y_f32 = fuse->y_f32;
+    *combined = true;
+  }
   // the down GEMM's TMA stores: o as [splits x split rows][d] fp32 (a caller's unsplit buffer
   // has exactly o_rows rows)
   CUtensorMap mo;
@@ -521,7 +578,7 @@ int moe_route_topk(const moe_dims* dims, const uint16_t* hidden, const float* ro
   if (router_uses_gemv(p)) {
     MOE_CUDA(cudaMemsetAsync(w.status + 3, 0, sizeof(int), s));   // the last-block counter
     MOE_CUDA(launch_route_gemv(p, hidden, router_w, router_bias, k, k_per_token, w.part, topk_ids,
-                               topk_w, nullptr, nullptr, false, w.status, s));
+                               topk_w, nullptr, nullptr, false, w.status, DecodeGrouping{}, s));
     return MOE_OK;
   }
   MOE_TRY(run_router_logits(p, w, hidden, router_w, s));
@@ -547,7 +604,7 @@ int moe_permute(const moe_dims* dims, const int32_t* topk_ids, int32_t k,
   q.shared = false;
   q.G = p.E;
   MOE_CUDA(launch_permute(q, topk_ids, k, k_per_token, expert_offsets, perm_token, inv_row,
-                          w.tiles, w.pscr, nullptr, w.status, static_cast<cudaStream_t>(stream)));
+                          w.tiles, w.pscr, w.status, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 
@@ -584,8 +641,10 @@ int moe_grouped_ffn_fp8(const moe_dims* dims, const uint16_t* hidden, const uint
   MOE_CUDA(cudaMemcpyAsync(w.perm, perm_token, sizeof(int32_t) * q.Rcap, cudaMemcpyDeviceToDevice, s));
   MOE_CUDA(cudaMemsetAsync(w.amax, 0, sizeof(uint32_t) * q.Rcap, s));   // the requant's row maxima
   const bool direct = p.g2_splits == 1;
+  bool combined = false;
   MOE_TRY(run_ffn(q, w, w13, w13_scale, w2, w2_scale, nullptr, nullptr, nullptr, nullptr,
-                  direct ? expert_out : w.o, (size_t)p.Rpad * p.d, q.Rcap, nullptr, s));
+                  direct ? expert_out : w.o, (size_t)p.Rpad * p.d, q.Rcap, nullptr, s, nullptr,
+                  &combined));
   if (!direct)
     MOE_CUDA(launch_reduce_splits(q, w.o, p.g2_splits, (size_t)p.Rpad * p.d, w.offsets + p.E,
                                   expert_out, s));
@@ -639,7 +698,8 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
     if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
   };
 
-  MOE_CUDA(cudaMemsetAsync(w.status, 0, 16, s));
+  // the status word and the counters of the fused decode epilogues
+  MOE_CUDA(cudaMemsetAsync(w.status, 0, p.off_counters + sizeof(int) * (size_t)std::max(p.n_tiles_cap, p.g2_m_tiles), s));
   record(0);
   if (router_is_fused(p)) {
     // one kernel for stages 0 and 1 (stage 1's events bracket nothing)
@@ -647,9 +707,11 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                                 w.xs, true, w.status, s));
     record(1);
   } else if (router_uses_gemv(p)) {
-    // decode batch: logits, top-k and quantisation in one kernel (stage 1's events bracket nothing)
+    // decode batch: logits, top-k, quantisation and the grouping in one kernel (the events of
+    // stages 1 and 2 bracket nothing)
+    const DecodeGrouping grp{w.offsets, w.perm, w.inv, w.tiles, w.amax, p.BN, p.shared ? 1 : 0};
     MOE_CUDA(launch_route_gemv(p, hidden, router_w, router_bias, k, k_per_token, w.part, w.ids,
-                               w.w, w.xq, w.xs, true, w.status, s));
+                               w.w, w.xq, w.xs, true, w.status, grp, s));
     record(1);
   } else {
     MOE_TRY(run_router_logits(p, w, hidden, router_w, s));
@@ -659,15 +721,29 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                                w.status, s));
   }
   record(2);
-  MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
-                          w.amax, w.status, s));
+  // grouping: by the decode router itself (T <= 8), alone (decode tiles: the gate/up GEMM fetches
+  // the rows), with the row gather in one kernel (prefill tiles, T * k_max <= 8192), or followed
+  // by the gather kernel
+  bool gathered = false;
+  if (router_uses_gemv(p)) {
+  } else if (p.BN <= 64 || !permute_gather_fused(p)) {
+    MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
+                            w.status, s));
+  } else {
+    MOE_CUDA(launch_permute_gather(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles,
+                                   w.xq, w.xs, w.xqp, w.xsp, w.amax, w.status, s));
+    gathered = true;
+  }
   const size_t split_stride = (size_t)p.Rpad * p.d;
+  const CombineOut cout{w.w, w.inv, y, dbg ? dbg->y_f32 : nullptr};
+  bool combined = false;
   MOE_TRY(run_ffn(p, w, w13, w13_scale, w2, w2_scale, w13_shared, w13s_scale, w2_shared,
-                  w2s_scale, w.o, split_stride, p.Rcap, ev, s));
+                  w2s_scale, w.o, split_stride, p.Rcap, ev, s, &cout, &combined, gathered));
   record(7);
-  MOE_CUDA(launch_combine(p, w.o, p.g2_splits, split_stride, w.w, w.inv,
-                          p.shared ? w.o : nullptr, p.shared ? w.offsets + p.E : nullptr,
-                          p.g2_splits, y, dbg ? dbg->y_f32 : nullptr, s));
+  if (!combined)
+    MOE_CUDA(launch_combine(p, w.o, p.g2_splits, split_stride, w.w, w.inv,
+                            p.shared ? w.o : nullptr, p.shared ? w.offsets + p.E : nullptr,
+                            p.g2_splits, y, dbg ? dbg->y_f32 : nullptr, s));
   record(8);
   if (dbg) {
     const size_t kk = (size_t)p.T * p.k_max;

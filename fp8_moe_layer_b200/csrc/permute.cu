@@ -1,8 +1,10 @@
 // Grouping of the routed (token, slot) pairs by expert: per-warp histograms, an exclusive prefix
-// sum over experts, and a stable scatter so routed rows are ordered by (expert, token). (The
-// grouped gate/up GEMM then fetches each routed row's token from the quantised hidden states
-// through perm; no row is copied.) The grouping also zeroes the row maxima of the SwiGLU output
-// that the gate/up GEMM accumulates with atomicMax.
+// sum over experts, and a stable scatter so routed rows are ordered by (expert, token). Then, for
+// prefill-sized token tiles, the gather that lays the quantised token rows out in that order for
+// the grouped GEMMs. (Decode-sized tiles skip it: their gate/up GEMM fetches the few rows of a tile
+// through the permutation with tile::gather4 loads. At prefill those four-row loads -- 32 per
+// pipeline stage of a 256-token tile -- made the GEMM TMA-issue-bound: 7650 vs 2659 us at
+// DeepSeek T=8192, so a gathered copy it is.)
 //
 // Method: "Routage MoE entre GPU" (viite.ai) -- only the selected experts process a token; the
 // tokens are dispatched to their experts and their order restored at the combine.
@@ -48,15 +50,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int& 
 // One block computes the whole grouping. Warp w owns tokens [w*chunk, (w+1)*chunk) and walks its
 // (token, slot) pairs in token-major order, 32 at a time. Lanes holding the same expert find each
 // other with __match_any_sync; a lane's rank among them plus the warp's running cursor for that
-// expert gives its row, so rows inside an expert are in ascending token order. Stores offsets,
-// perm, inv and the GEMM tile prefix, reports bad ids, zeroes amax[r] of every routed (and
-// shared) row when amax is given, and returns the routed row count R.
+// expert gives its row, so rows inside an expert are in ascending token order. `write` selects
+// the block that stores offsets / perm / inv / tiles (and reports bad ids); `s_perm`, when given,
+// receives perm[] in shared memory. Returns the routed row count R.
 __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_max, int k,
                                   const int32_t* __restrict__ k_per_token, int E, int has_shared,
                                   int BN, int32_t* __restrict__ offsets,
                                   int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                                   int32_t* __restrict__ tiles, int* status, int* hist,
-                                  int* warp_sums, uint32_t* __restrict__ amax) {
+                                  int* warp_sums, int* s_perm, bool write) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kPermWarps * E; i += kPermThreads) hist[i] = 0;
   __syncthreads();
@@ -75,7 +77,7 @@ __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_
       if (j < kt) {
         const int e = ids[idx];
         if (e >= 0 && e < E) atomicAdd(&my_hist[e], 1);
-        else report(status, kStatusDeviceCheck, kWherePermute, t);
+        else if (write) report(status, kStatusDeviceCheck, kWherePermute, t);
       }
     }
   }
@@ -90,7 +92,7 @@ __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_
       for (int w = 0; w < kPermWarps; ++w) cnt += hist[w * E + e];
     const int off = block_exclusive_scan(cnt, warp_sums, total_rows);
     if (e < E) {
-      offsets[e] = off;
+      if (write) offsets[e] = off;
       int run = off;
       for (int w = 0; w < kPermWarps; ++w) {
         const int c = hist[w * E + e];
@@ -100,8 +102,8 @@ __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_
     }
     const int nt = e < E ? (cnt + BN - 1) / BN : 0;
     const int toff = block_exclusive_scan(nt, warp_sums, total_tiles);
-    if (e < E) tiles[e] = toff;
-    if (threadIdx.x == 0) {
+    if (write && e < E) tiles[e] = toff;
+    if (write && threadIdx.x == 0) {
       offsets[E] = total_rows;
       if (has_shared) {
         offsets[E + 1] = total_rows + T;
@@ -127,7 +129,7 @@ __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_
         e = ids[idx];
         valid = e >= 0 && e < E;
       }
-      if (!valid) inv[idx] = -1;
+      if (!valid && write) inv[idx] = -1;
     }
     const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : E + lane);
     const int rank = __popc(peers & ((1u << lane) - 1u));
@@ -135,17 +137,19 @@ __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_
     __syncwarp();
     if (valid) {
       const int r = cursor + rank;
-      perm[r] = t;
-      inv[idx] = r;
-      if (amax) amax[r] = 0u;
+      if (write) {
+        perm[r] = t;
+        inv[idx] = r;
+      }
+      if (s_perm) s_perm[r] = t;
       if (rank == 0) my_hist[e] = cursor + __popc(peers);
     }
     __syncwarp();
   }
   if (has_shared)
     for (int t = threadIdx.x; t < T; t += kPermThreads) {
-      perm[total_rows + t] = t;
-      if (amax) amax[total_rows + t] = 0u;
+      if (write) perm[total_rows + t] = t;
+      if (s_perm) s_perm[total_rows + t] = t;
     }
   return total_rows;
 }
@@ -153,14 +157,49 @@ __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(
     const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
     int E, int has_shared, int BN, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
-    int32_t* __restrict__ inv, int32_t* __restrict__ tiles, uint32_t* __restrict__ amax,
-    int* status) {
+    int32_t* __restrict__ inv, int32_t* __restrict__ tiles, int* status) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   extern __shared__ int hist[];                  // [kPermWarps][E]
   __shared__ int warp_sums[33];
   permute_block_body(ids, T, k_max, k, k_per_token, E, has_shared, BN, offsets, perm, inv, tiles,
-                     status, hist, warp_sums, amax);
+                     status, hist, warp_sums, nullptr, true);
+}
+
+// Grouping and row gather in one kernel, for batches whose grouping fits one block (T * k_max <=
+// 8192): every block computes the (small) grouping itself into shared memory -- so no block
+// waits for another -- block 0 also stores it, and each block then copies its share of the
+// quantised token rows into grouped order (one warp per row): xqp[r, :] = xq[perm[r], :],
+// xsp[r] = xs[perm[r]], amax[r] = 0. Saves the separate gather launch and its dependency wait.
+__global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(
+    const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
+    int E, int has_shared, int BN, int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv, int32_t* __restrict__ tiles, const uint8_t* __restrict__ xq,
+    const float* __restrict__ xs, int d, uint8_t* __restrict__ xqp, float* __restrict__ xsp,
+    uint32_t* __restrict__ amax, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  extern __shared__ int smem_i[];                // hist [kPermWarps][E], then perm [rows]
+  __shared__ int warp_sums[33];
+  int* hist = smem_i;
+  int* s_perm = smem_i + kPermWarps * E;
+  const int R = permute_block_body(ids, T, k_max, k, k_per_token, E, has_shared, BN, offsets, perm,
+                                   inv, tiles, status, hist, warp_sums, s_perm, blockIdx.x == 0);
+  __syncthreads();
+  const int rows = R + (has_shared ? T : 0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nv = d / 16;
+  for (int r = blockIdx.x * kPermWarps + warp; r < rows; r += gridDim.x * kPermWarps) {
+    const int t = s_perm[r];
+    const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xqp + (size_t)r * d);
+#pragma unroll 4
+    for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+    if (lane == 0) {
+      xsp[r] = xs[t];
+      amax[r] = 0u;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -260,7 +299,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_scan_kernel(
 __global__ void __launch_bounds__(kPermBlkThreads) permute_scatter_kernel(
     const int32_t* __restrict__ ids, int T, int k_max, int k, const int32_t* __restrict__ k_per_token,
     int E, int has_shared, const int32_t* __restrict__ bbase, const int32_t* __restrict__ offsets,
-    int32_t* __restrict__ perm, int32_t* __restrict__ inv, uint32_t* __restrict__ amax) {
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   extern __shared__ int whist[];
@@ -301,17 +340,14 @@ __global__ void __launch_bounds__(kPermBlkThreads) permute_scatter_kernel(
       const int r = cursor + rank;
       perm[r] = t;
       inv[idx] = r;
-      if (amax) amax[r] = 0u;
       if (rank == 0) my[e] = cursor + __popc(peers);
     }
     __syncwarp();
   }
   if (has_shared) {
     const int R = offsets[E];
-    for (int t = blockIdx.x * kPermBlkThreads + threadIdx.x; t < T; t += gridDim.x * kPermBlkThreads) {
+    for (int t = blockIdx.x * kPermBlkThreads + threadIdx.x; t < T; t += gridDim.x * kPermBlkThreads)
       perm[R + t] = t;
-      if (amax) amax[R + t] = 0u;
-    }
   }
 }
 
@@ -345,6 +381,37 @@ __global__ void __launch_bounds__(kPermThreads) tile_prefix_kernel(
   if (threadIdx.x == 0) tiles[E] = total;
 }
 
+// One warp per routed row: xqp[r, :] = xq[perm[r], :], xsp[r] = xs[perm[r]], amax[r] = 0.
+// A token index outside [0, T) (caller-provided permutation) gives a zero row and flags
+// MOE_ERR_DEVICE_CHECK.
+__global__ void __launch_bounds__(256) gather_rows_kernel(
+    const uint8_t* __restrict__ xq, const float* __restrict__ xs, const int32_t* __restrict__ perm,
+    const int32_t* __restrict__ total_rows, int64_t rcap, int T, int d, uint8_t* __restrict__ xqp,
+    float* __restrict__ xsp, uint32_t* __restrict__ amax, int* status) {
+  pdl_wait();      // predecessor kernel complete, its writes visible
+  pdl_trigger();   // let the next kernel launch
+  const int R = (int)min((int64_t)max(*total_rows, 0), rcap);
+  const int lane = threadIdx.x & 31;
+  const int nv = d / 16;
+  for (int r = blockIdx.x * 8 + (threadIdx.x >> 5); r < R; r += gridDim.x * 8) {
+    const int t = perm[r];
+    const bool ok = t >= 0 && t < T;
+    uint4* dst = reinterpret_cast<uint4*>(xqp + (size_t)r * d);
+    if (ok) {
+      const uint4* src = reinterpret_cast<const uint4*>(xq + (size_t)t * d);
+#pragma unroll 4
+      for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+    } else {
+      for (int i = lane; i < nv; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (lane == 0) {
+      xsp[r] = ok ? xs[t] : 0.f;
+      amax[r] = 0u;
+      if (!ok) report(status, kStatusDeviceCheck, kWhereGather, r);
+    }
+  }
+}
+
 // Blocks of the multi-block grouping: about 1024 (token, slot) pairs each, at most 4 per SM.
 int permute_blocks(const Plan& p) {
   const long long slots = (long long)p.T * p.k_max;
@@ -354,7 +421,7 @@ int permute_blocks(const Plan& p) {
 
 cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32_t* k_per_token,
                            int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* tiles,
-                           int32_t* scratch, uint32_t* amax, int* status, cudaStream_t s) {
+                           int32_t* scratch, int* status, cudaStream_t s) {
   const int blocks = permute_blocks(p);
   if (blocks == 1) {
     const size_t smem = sizeof(int) * kPermWarps * p.E;
@@ -370,7 +437,7 @@ cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32
     }
     launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), smem, s, ids, p.T, p.k_max, k, k_per_token, p.E,
                                                  p.shared ? 1 : 0, p.BN, offsets, perm, inv, tiles,
-                                                 amax, status);
+                                                 status);
     return cudaGetLastError();
   }
   int32_t* bcount = scratch;
@@ -382,7 +449,35 @@ cudaError_t launch_permute(const Plan& p, const int32_t* ids, int k, const int32
                                                  bbase, offsets, tiles);
   launch_pdl(permute_scatter_kernel, dim3(blocks), dim3(kPermBlkThreads), smem, s, ids, p.T, p.k_max, k, k_per_token,
                                                                p.E, p.shared ? 1 : 0, bbase,
-                                                               offsets, perm, inv, amax);
+                                                               offsets, perm, inv);
+  return cudaGetLastError();
+}
+
+bool permute_gather_fused(const Plan& p) { return permute_blocks(p) == 1; }
+
+cudaError_t launch_permute_gather(const Plan& p, const int32_t* ids, int k,
+                                  const int32_t* k_per_token, int32_t* offsets, int32_t* perm,
+                                  int32_t* inv, int32_t* tiles, const uint8_t* xq, const float* xs,
+                                  uint8_t* xqp, float* xsp, uint32_t* amax, int* status,
+                                  cudaStream_t s) {
+  // T * k_max <= 8192 here, so rows = T * k_max (+ T) <= 16384
+  const size_t smem = sizeof(int) * ((size_t)kPermWarps * p.E + (size_t)p.Rcap);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(permute_gather_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(int) * (kPermWarps * kMaxExperts + 16384));
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  // about 32 KB of rows per block (one warp per row), at most one block per SM
+  const int64_t bytes = p.Rcap * (int64_t)p.d;
+  const int grid = (int)std::min<int64_t>(std::max<int64_t>((bytes + 32767) / 32768, 1), num_sms());
+  launch_pdl(permute_gather_kernel, dim3(grid), dim3(kPermThreads), smem, s, ids, p.T, p.k_max, k,
+             k_per_token, p.E, p.shared ? 1 : 0, p.BN, offsets, perm, inv, tiles, xq, xs, p.d,
+             xqp, xsp, amax, status);
   return cudaGetLastError();
 }
 
@@ -390,6 +485,16 @@ cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* t
                                cudaStream_t s) {
   launch_pdl(tile_prefix_kernel, dim3(1), dim3(kPermThreads), 0, s, offsets, p.E, (int64_t)p.T * p.k_max, p.BN, tiles,
                                                 status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, const int32_t* perm,
+                          const int32_t* total_rows, uint8_t* xqp, float* xsp, uint32_t* amax,
+                          int* status, cudaStream_t s) {
+  const int64_t blocks_needed = (p.Rcap + 7) / 8;
+  const int grid = (int)std::min<int64_t>(std::max<int64_t>(blocks_needed, 1), 8LL * num_sms());
+  launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, s, xq, xs, perm, total_rows, p.Rcap, p.T, p.d, xqp, xsp,
+                                          amax, status);
   return cudaGetLastError();
 }
 

@@ -19,6 +19,8 @@
 // tensor-core logits (router_mma.cu) are only a filter: the experts they leave in play are
 // recomputed in fp64 before the selection. The weights exp(l_j - l_max) / sum are computed in fp64
 // and rounded once to fp32.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -148,15 +150,27 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 //         renormalised over the selection.
 //  quant: s_t = amax|x[t,:]| / 448 (IEEE fp32 division; 1 if amax = 0);
 //         xq = e4m3_rne_satfinite(x / s_t) (IEEE fp32 division).
+//  refine (refine_w != null, for the tensor-core logits): the approximate logits only pick the
+//         candidates -- every expert within kRefineWindow of the approximate k_t-th largest, which
+//         contains the exact top-k_t while the approximation error stays below half the window --
+//         and each candidate's logit is recomputed in fp64 (one warp per candidate) before the
+//         selection and the weights.
+constexpr double kRefineWindow = 1e-2;
+constexpr int kMaxCandidates = 256;
+
 __global__ void __launch_bounds__(128) topk_quant_kernel(
     const double* __restrict__ part, int splits, const float* __restrict__ bias, int T, int E,
     int k, const int32_t* __restrict__ k_per_token, int k_max, int32_t* __restrict__ ids,
     float* __restrict__ wout, const uint16_t* __restrict__ x, int d, uint8_t* __restrict__ xq,
-    float* __restrict__ xs, int do_route, int do_quant, int* status) {
+    float* __restrict__ xs, int do_route, int do_quant, const float* __restrict__ refine_w,
+    int* status) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   __shared__ double lg[kMaxExperts];
   __shared__ float red[4];
+  __shared__ int cand[kMaxCandidates];
+  __shared__ int ncand;
+  __shared__ double vk_s;
   const int t = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -182,10 +196,52 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
       if (tid == 0) report(status, kStatusDeviceCheck, kWhereRoute, t);
       kt = max(1, min(kt, kcap));
     }
+    bool by_cand = false;          // exact selection over the refined candidates only
+    if (refine_w) {
+      if (warp == 0) {
+        double sv;
+        int se;
+        warp_select_desc(E, kt, [&](int c) { return lg[c]; }, [](int c) { return c; }, sv, se);
+        const double vk = __shfl_sync(0xffffffffu, sv, kt - 1);   // approximate k_t-th largest
+        if (lane == 0) {
+          vk_s = vk;
+          ncand = 0;
+        }
+      }
+      __syncthreads();
+      const double floor_v = vk_s - kRefineWindow;
+      for (int e = tid; e < E; e += 128) {
+        if (lg[e] >= floor_v) {
+          const int c = atomicAdd(&ncand, 1);
+          if (c < kMaxCandidates) cand[c] = e;
+        }
+      }
+      __syncthreads();
+      const bool all = ncand > kMaxCandidates;          // pathological: recompute every expert
+      const int nc = all ? E : ncand;
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+      const int nv = d / 8;
+      for (int c = warp; c < nc; c += 4) {
+        const int e = all ? c : cand[c];
+        const float4* wr = reinterpret_cast<const float4*>(refine_w + (size_t)e * d);
+        double acc = 0.0;
+#pragma unroll 4
+        for (int i = lane; i < nv; i += 32) acc += dot8_f64(xr[i], __ldg(wr + 2 * i), __ldg(wr + 2 * i + 1));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) lg[e] = acc + (bias ? static_cast<double>(bias[e]) : 0.0);
+      }
+      __syncthreads();
+      by_cand = !all;
+    }
     if (warp == 0) {
       double sv;
       int se;
-      warp_select_desc(E, kt, [&](int c) { return lg[c]; }, [](int c) { return c; }, sv, se);
+      if (by_cand)
+        warp_select_desc(ncand, kt, [&](int c) { return lg[cand[c]]; },
+                         [&](int c) { return cand[c]; }, sv, se);
+      else
+        warp_select_desc(E, kt, [&](int c) { return lg[c]; }, [](int c) { return c; }, sv, se);
       warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
     }
   }
@@ -229,240 +285,6 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
   }
 }
 
-// FP8 e4m3 quantisation of one token row by one warp: s = amax|x| / 448 (IEEE fp32; 1 if 0),
-// code = e4m3_rne_satfinite(x / s) (IEEE fp32 division).
-__device__ __forceinline__ void warp_quant_row(const uint16_t* __restrict__ xrow, int d,
-                                               uint8_t* __restrict__ qrow, float* __restrict__ s_out) {
-  const int lane = threadIdx.x & 31;
-  const uint4* xr = reinterpret_cast<const uint4*>(xrow);
-  const int nv = d / 8;
-  float amax = 0.f;
-  for (int i = lane; i < nv; i += 32) {
-    const uint4 v = xr[i];
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w4[q] << 16)),
-                               fabsf(__uint_as_float(w4[q] & 0xFFFF0000u))));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-  if (lane == 0) *s_out = sc;
-  uint2* out = reinterpret_cast<uint2*>(qrow);
-  for (int i = lane; i < nv; i += 32) {
-    const uint4 v = xr[i];
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-    uint32_t packed[2];
-#pragma unroll
-    for (int q = 0; q < 4; q += 2) {
-      const float a0 = __fdiv_rn(__uint_as_float(w4[q] << 16), sc);
-      const float a1 = __fdiv_rn(__uint_as_float(w4[q] & 0xFFFF0000u), sc);
-      const float a2 = __fdiv_rn(__uint_as_float(w4[q + 1] << 16), sc);
-      const float a3 = __fdiv_rn(__uint_as_float(w4[q + 1] & 0xFFFF0000u), sc);
-      packed[q / 2] = static_cast<uint32_t>(e4m3x2(a0, a1)) |
-                      (static_cast<uint32_t>(e4m3x2(a2, a3)) << 16);
-    }
-    out[i] = make_uint2(packed[0], packed[1]);
-  }
-}
-
-// Selection after the tensor-core logits (router_mma.cu), for blocks of kRfTok tokens (256
-// threads; warp w owns the block's tokens w, w + 8, ...):
-//  1. candidates: each token's approximate logits (tensor-core sum + bias) pick every expert
-//     within kRefineWindow of the approximate k_t-th largest -- which contains the exact top-k_t
-//     while the approximation error stays below half the window -- into the block's list of
-//     (token, expert) pairs, sorted by expert with a counting sort;
-//  2. exact logits of the pairs in fp64, d in chunks of kRfChunk: the block's hidden rows of a
-//     chunk sit in shared memory, and the warps walk the pairs in expert order, so each
-//     expert's weight chunk is fetched from L2 about once per block, not once per token;
-//  3. selection (descending, exact ties to the lower id) and weights from the exact logits;
-//  4. the tokens' FP8 quantisation (when asked).
-// A token with more than kRfCandTok candidates (near-equal logits everywhere, e.g. a zero row)
-// has all E logits recomputed exactly by its warp instead, into the `approx` buffer.
-constexpr double kRefineWindow = 1e-2;
-constexpr int kRfTok = 32;
-constexpr int kRfChunk = 1024;
-constexpr int kRfCandTok = 64;
-constexpr int kRfPairs = kRfTok * kRfCandTok;
-constexpr int kRfSmem = kRfTok * kRfChunk * 2 + kRfPairs * (4 + 8 + 2) + (kMaxExperts + 1) * 4;
-
-__global__ void __launch_bounds__(256) route_refine_kernel(
-    double* __restrict__ approx, const float* __restrict__ bias, int T, int E, int k,
-    const int32_t* __restrict__ k_per_token, int k_max, int32_t* __restrict__ ids,
-    float* __restrict__ wout, const uint16_t* __restrict__ x, int d,
-    const float* __restrict__ W, uint8_t* __restrict__ xq, float* __restrict__ xs, int do_quant,
-    int* status) {
-  pdl_wait();      // predecessor kernel complete, its writes visible
-  pdl_trigger();   // let the next kernel launch
-  extern __shared__ __align__(16) uint8_t rf_smem[];
-  uint16_t* xsm = reinterpret_cast<uint16_t*>(rf_smem);                   // [kRfTok][kRfChunk]
-  int* pairs = reinterpret_cast<int*>(rf_smem + kRfTok * kRfChunk * 2);   // (token << 16) | e
-  double* acc = reinterpret_cast<double*>(pairs + kRfPairs);              // exact logit sums
-  uint16_t* order = reinterpret_cast<uint16_t*>(acc + kRfPairs);          // pairs by expert
-  int* hist = reinterpret_cast<int*>(order + kRfPairs);                   // [E + 1]
-  __shared__ int tok_start[kRfTok], tok_n[kRfTok], tok_kt[kRfTok];
-  __shared__ int np_s;
-  __shared__ int warp_sums[9];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = blockIdx.x * kRfTok;
-  const int kcap = min(E, k_max);
-  if (tid == 0) np_s = 0;
-  for (int e = tid; e <= E; e += 256) hist[e] = 0;
-  __syncthreads();
-
-  // ---- 1. candidates (each warp stages its token's approximate logits in its slice of xsm)
-  double* lrow = reinterpret_cast<double*>(xsm) + warp * kMaxExperts;
-  for (int tl = warp; tl < kRfTok; tl += 8) {
-    const int t = t0 + tl;
-    if (t >= T) {
-      if (lane == 0) tok_n[tl] = 0;
-      continue;
-    }
-    int kt = k_per_token ? k_per_token[t] : k;
-    if (kt < 1 || kt > kcap) {
-      if (lane == 0) report(status, kStatusDeviceCheck, kWhereRoute, t);
-      kt = max(1, min(kt, kcap));
-    }
-    for (int e = lane; e < E; e += 32)
-      lrow[e] = approx[(size_t)t * E + e] + (bias ? static_cast<double>(bias[e]) : 0.0);
-    __syncwarp();
-    double sv;
-    int se;
-    warp_select_desc(E, kt, [&](int c) { return lrow[c]; }, [](int c) { return c; }, sv, se);
-    const double floor_v = __shfl_sync(0xffffffffu, sv, kt - 1) - kRefineWindow;
-    int n = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      n += __popc(__ballot_sync(0xffffffffu, e < E && lrow[e] >= floor_v));
-    }
-    int start = 0;
-    if (n <= kRfCandTok) {
-      if (lane == 0) start = atomicAdd(&np_s, n);
-      start = __shfl_sync(0xffffffffu, start, 0);
-      int pos = start;
-      for (int e0 = 0; e0 < E; e0 += 32) {
-        const int e = e0 + lane;
-        const bool in = e < E && lrow[e] >= floor_v;
-        const unsigned m = __ballot_sync(0xffffffffu, in);
-        if (in) {
-          const int p = pos + __popc(m & ((1u << lane) - 1u));
-          pairs[p] = (tl << 16) | e;
-          acc[p] = 0.0;
-          atomicAdd(&hist[e], 1);
-        }
-        pos += __popc(m);
-      }
-    }
-    if (lane == 0) {
-      tok_start[tl] = start;
-      tok_n[tl] = n <= kRfCandTok ? n : -1;       // -1: every expert recomputed (step 3)
-      tok_kt[tl] = kt;
-    }
-    __syncwarp();
-  }
-  __syncthreads();
-  const int np = np_s;
-  // counting sort of the pairs by expert: exclusive prefix of hist over E (one pass per thread
-  // over a contiguous range of experts, then a scan of the 256 range totals)
-  {
-    const int per = (E + 255) / 256;
-    const int e_lo = min(E, tid * per), e_hi = min(E, e_lo + per);
-    int run = 0;
-    for (int e = e_lo; e < e_hi; ++e) run += hist[e];
-    int incl = run;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (tid == 0) {
-      int s = 0;
-      for (int w = 0; w < 8; ++w) {
-        const int v = warp_sums[w];
-        warp_sums[w] = s;
-        s += v;
-      }
-    }
-    __syncthreads();
-    int base = warp_sums[warp] + incl - run;
-    for (int e = e_lo; e < e_hi; ++e) {
-      const int c = hist[e];
-      hist[e] = base;
-      base += c;
-    }
-  }
-  __syncthreads();
-  for (int p = tid; p < np; p += 256) {
-    const int e = pairs[p] & 0xFFFF;
-    order[atomicAdd(&hist[e], 1)] = static_cast<uint16_t>(p);
-  }
-  __syncthreads();
-
-  // ---- 2. exact logits of the pairs, chunk by chunk of d (lane l takes the 8-element groups
-  //         l, l + 32, ... of the chunk: conflict-free shared loads, coalesced weight loads)
-  for (int c0 = 0; c0 < d; c0 += kRfChunk) {
-    const int cw = min(kRfChunk, d - c0);           // a multiple of 16
-    const int nv = cw / 8;
-    for (int i = tid; i < kRfTok * (kRfChunk / 8); i += 256) {
-      const int tl = i / (kRfChunk / 8), v = i % (kRfChunk / 8);
-      const int t = t0 + tl;
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      if (t < T && v < nv) val = reinterpret_cast<const uint4*>(x + (size_t)t * d + c0)[v];
-      reinterpret_cast<uint4*>(xsm)[i] = val;
-    }
-    __syncthreads();
-    for (int i = warp; i < np; i += 8) {
-      const int p = order[i];
-      const int tl = pairs[p] >> 16, e = pairs[p] & 0xFFFF;
-      const uint4* xr = reinterpret_cast<const uint4*>(xsm + tl * kRfChunk);
-      const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d + c0);
-      double part = 0.0;
-#pragma unroll 4
-      for (int v = lane; v < nv; v += 32) part += dot8_f64(xr[v], __ldg(wr + 2 * v), __ldg(wr + 2 * v + 1));
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      if (lane == 0) acc[p] += part;
-    }
-    __syncthreads();
-  }
-
-  // ---- 3. selection from the exact logits, 4. quantisation
-  for (int tl = warp; tl < kRfTok; tl += 8) {
-    const int t = t0 + tl;
-    if (t >= T) continue;
-    const int kt = tok_kt[tl], n = tok_n[tl], start = tok_start[tl];
-    double sv;
-    int se;
-    if (n >= 0) {
-      warp_select_desc(n, kt,
-                       [&](int c) {
-                         const int e = pairs[start + c] & 0xFFFF;
-                         return acc[start + c] + (bias ? static_cast<double>(bias[e]) : 0.0);
-                       },
-                       [&](int c) { return pairs[start + c] & 0xFFFF; }, sv, se);
-    } else {
-      double* row = approx + (size_t)t * E;
-      const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-      for (int e = 0; e < E; ++e) {
-        const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
-        double a = 0.0;
-        for (int v = lane; v < d / 8; v += 32) a += dot8_f64(xr[v], __ldg(wr + 2 * v), __ldg(wr + 2 * v + 1));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
-        if (lane == 0) row[e] = a + (bias ? static_cast<double>(bias[e]) : 0.0);
-      }
-      __syncwarp();
-      warp_select_desc(E, kt, [&](int c) { return __ldcg(row + c); }, [](int c) { return c; },
-                       sv, se);
-    }
-    warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
-    if (do_quant) warp_quant_row(x + (size_t)t * d, d, xq + (size_t)t * d, xs + t);
-  }
-}
-
 // Decode router (T <= 8 tokens, E > 32): one warp per expert computes that expert's fp64 logit
 // for every token (lane-strided chunks of 8 along d, then a butterfly; all loads in flight),
 // writes it to `logits` [T][E], and the last block to finish (a counter in the status word,
@@ -472,12 +294,41 @@ __global__ void __launch_bounds__(256) route_refine_kernel(
 // block's copy of the logits).
 constexpr int kGemvMaxT = 8;
 
+// Exclusive prefix sum over the 256 threads of a block (tmp: 9 ints of shared memory); returns
+// this thread's exclusive prefix and the block total in `total`.
+__device__ __forceinline__ int block_exscan256(int v, int* tmp, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int w = 0; w < 8; ++w) {
+      const int c = tmp[w];
+      tmp[w] = s;
+      s += c;
+    }
+    tmp[8] = s;
+  }
+  __syncthreads();
+  const int r = tmp[warp] + incl - v;
+  total = tmp[8];
+  __syncthreads();
+  return r;
+}
+
 template <int TT>
 __global__ void __launch_bounds__(256) route_gemv_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ W, const float* __restrict__ bias,
     int T, int d, int E, int k, const int32_t* __restrict__ k_per_token, int k_max,
     double* __restrict__ logits, int32_t* __restrict__ ids, float* __restrict__ wout,
-    uint8_t* __restrict__ xq, float* __restrict__ xs, int do_quant, int* status) {
+    uint8_t* __restrict__ xq, float* __restrict__ xs, int do_quant, int* status,
+    const DecodeGrouping grp) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
   __shared__ int s_last;
@@ -529,6 +380,77 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
     int se;
     warp_select_desc(E, kt, [&](int c) { return my[c]; }, [](int c) { return c; }, sv, se);
     warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
+  }
+  if (grp.offsets) {
+    // The grouping of the (at most 8 x 32) routed pairs, by this block: expert counts, their
+    // exclusive prefix (offsets), each pair's row = offset + its rank among the earlier pairs of
+    // the same expert (token-major order: stable), and the GEMM tile prefix. Same result as the
+    // grouping kernels (permute.cu); it also zeroes the rows' SwiGLU maxima.
+    __syncthreads();                                   // ids of every token written
+    __shared__ int tmp[9];
+    int* cnt = reinterpret_cast<int*>(lgd);            // [E] (the logit copies are done with)
+    int* off = cnt + E;                                // [E]
+    for (int e = tid; e < E; e += 256) cnt[e] = 0;
+    __syncthreads();
+    const int npairs = T * k_max;                      // <= 8 * 32 = 256 = blockDim
+    int my_e = -1;
+    if (tid < npairs) {
+      const int t = tid / k_max, j = tid % k_max;
+      int kt = k_per_token ? k_per_token[t] : k;
+      kt = max(1, min(kt, min(E, k_max)));
+      const int e = j < kt ? ids[tid] : -1;
+      if (e >= 0 && e < E) {
+        my_e = e;
+        atomicAdd(&cnt[e], 1);
+      }
+    }
+    __syncthreads();
+    const int per = (E + 255) / 256;
+    const int e_lo = min(E, tid * per), e_hi = min(E, e_lo + per);
+    int seg = 0, seg_tiles = 0;
+    for (int e = e_lo; e < e_hi; ++e) {
+      seg += cnt[e];
+      seg_tiles += (cnt[e] + grp.BN - 1) / grp.BN;
+    }
+    int R = 0, total_tiles = 0;
+    int base = block_exscan256(seg, tmp, R);
+    int tbase = block_exscan256(seg_tiles, tmp, total_tiles);
+    for (int e = e_lo; e < e_hi; ++e) {
+      off[e] = base;
+      grp.offsets[e] = base;
+      grp.tiles[e] = tbase;
+      base += cnt[e];
+      tbase += (cnt[e] + grp.BN - 1) / grp.BN;
+    }
+    __syncthreads();
+    if (tid < npairs) {
+      int row = -1;
+      if (my_e >= 0) {
+        int rank = 0;
+        for (int i = 0; i < tid; ++i) {
+          const int ti = i / k_max, ji = i % k_max;
+          int kti = k_per_token ? k_per_token[ti] : k;
+          kti = max(1, min(kti, min(E, k_max)));
+          if (ji < kti && ids[i] == my_e) ++rank;
+        }
+        row = off[my_e] + rank;
+        grp.perm[row] = tid / k_max;
+        grp.amax[row] = 0u;
+      }
+      grp.inv[tid] = row;
+    }
+    if (tid == 0) {
+      grp.offsets[E] = R;
+      grp.tiles[E] = total_tiles;
+      if (grp.has_shared) {
+        grp.offsets[E + 1] = R + T;
+        grp.tiles[E + 1] = total_tiles + (T + grp.BN - 1) / grp.BN;
+      }
+    }
+    if (grp.has_shared && tid < T) {
+      grp.perm[R + tid] = tid;
+      grp.amax[R + tid] = 0u;
+    }
   }
   if (do_quant) {
     // the FP8 quantisation of each token by the whole block
@@ -717,32 +639,34 @@ template <int TT>
 static cudaError_t launch_gemv_t(const Plan& p, const uint16_t* hidden, const float* router_w,
                                  const float* bias, int k, const int32_t* k_per_token,
                                  double* logits, int32_t* ids, float* w, uint8_t* xq, float* xs,
-                                 int q, int* status, cudaStream_t s) {
+                                 int q, int* status, const DecodeGrouping& grp, cudaStream_t s) {
   static bool done[64] = {};
   cudaError_t err = allow_dynamic_smem(route_gemv_kernel<TT>, kGemvMaxT * kMaxExperts * 8, done);
   if (err != cudaSuccess) return err;
-  const size_t smem = sizeof(double) * (size_t)p.T * p.E;
+  // the logit copies of the last block; the grouping reuses it for two ints per expert
+  const size_t smem = std::max(sizeof(double) * (size_t)p.T * p.E, sizeof(int) * 2 * (size_t)p.E);
   launch_pdl(route_gemv_kernel<TT>, dim3((p.E + 7) / 8), dim3(256), smem, s, hidden, router_w,
-             bias, p.T, p.d, p.E, k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status);
+             bias, p.T, p.d, p.E, k, k_per_token, p.k_max, logits, ids, w, xq, xs, q, status, grp);
   return cudaGetLastError();
 }
 
 cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
                               const float* bias, int k, const int32_t* k_per_token,
                               double* logits, int32_t* ids, float* w, uint8_t* xq, float* xs,
-                              bool do_quant, int* status, cudaStream_t s) {
+                              bool do_quant, int* status, const DecodeGrouping& grp,
+                              cudaStream_t s) {
   const int q = do_quant ? 1 : 0;
   if (p.T <= 1)
     return launch_gemv_t<1>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
-                            status, s);
+                            status, grp, s);
   if (p.T <= 2)
     return launch_gemv_t<2>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
-                            status, s);
+                            status, grp, s);
   if (p.T <= 4)
     return launch_gemv_t<4>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
-                            status, s);
+                            status, grp, s);
   return launch_gemv_t<8>(p, hidden, router_w, bias, k, k_per_token, logits, ids, w, xq, xs, q,
-                          status, s);
+                          status, grp, s);
 }
 
 cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
@@ -754,22 +678,13 @@ cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const fl
   return cudaGetLastError();
 }
 
-cudaError_t launch_topk_quant(const Plan& p, double* part, const float* bias, int k,
+cudaError_t launch_topk_quant(const Plan& p, const double* part, const float* bias, int k,
                               const int32_t* k_per_token, int32_t* ids, float* w,
                               const uint16_t* hidden, uint8_t* xq, float* xs, bool do_route,
                               bool do_quant, const float* refine_w, int* status, cudaStream_t s) {
-  if (do_route && refine_w) {
-    static bool done[64] = {};
-    cudaError_t err = allow_dynamic_smem(route_refine_kernel, kRfSmem, done);
-    if (err != cudaSuccess) return err;
-    launch_pdl(route_refine_kernel, dim3((p.T + kRfTok - 1) / kRfTok), dim3(256), kRfSmem, s,
-               part, bias, p.T, p.E, k, k_per_token, p.k_max, ids, w, hidden, p.d, refine_w, xq,
-               xs, do_quant ? 1 : 0, status);
-    return cudaGetLastError();
-  }
   launch_pdl(topk_quant_kernel, dim3(p.T), dim3(128), 0, s, part, p.r_splits, bias, p.T, p.E, k,
              k_per_token, p.k_max, ids, w, hidden, p.d, xq, xs, do_route ? 1 : 0,
-             do_quant ? 1 : 0, status);
+             do_quant ? 1 : 0, refine_w, status);
   return cudaGetLastError();
 }
 
