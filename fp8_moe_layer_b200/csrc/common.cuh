@@ -191,21 +191,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// L2 prefetch of a tensor tile (no shared memory, no completion): the tile is on its way to L2
-// when the TMA load for it is issued later.
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int x, int y, int z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int x, int y, int z, int w) {
-  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(z), "r"(w)
-               : "memory");
-}
-
 // Loads issued by either CTA of a 2-CTA (cta_group::2) pair: the data lands in the issuing CTA's
 // shared memory, the transaction bytes are counted on the barrier at `bar` (a shared::cluster
 // address, here always the even CTA's barrier, which waits for both CTAs' bytes).

@@ -141,101 +141,6 @@ __device__ __forceinline__ int tile_rows_rounded(const TileTable& tt, int g, int
 }
 
 
-// ---------------------------------------------------------------- decode fusions (epilogue warps)
-// Both run on the 128 epilogue threads (e = threadIdx.x - 128) of the CTA that finished the last
-// tile of a token tile (SwiGLU) or of an output-channel tile (combine), after an acquire fence;
-// every read of another CTA's output goes through L2 (ld.global.cg).
-
-// Rows row0 .. row0 + nrows - 1 of the K-split gate/up partials h[s][r][2F] (scaled sums):
-// act = silu(sum_s gate) * sum_s up (split order fixed), s2[r] = amax|act| / 448 (IEEE fp32;
-// 1 if 0), aq[r] = e4m3(act / s2[r]). The same arithmetic as swiglu_requant_kernel.
-__device__ __forceinline__ void fused_swiglu_requant(const GemmArgs& a, int row0, int nrows,
-                                                     float* red) {
-  const int e = threadIdx.x - 128, lane = threadIdx.x & 31, q = e >> 5;
-  const int F = a.F, nv = F / 4;
-  for (int rr = 0; rr < nrows; ++rr) {
-    const int r = row0 + rr;
-    auto act4 = [&](int i) {
-      const float* hr = a.out + (size_t)r * a.out_ld;
-      float4 gv = __ldcg(reinterpret_cast<const float4*>(hr) + i);
-      float4 uv = __ldcg(reinterpret_cast<const float4*>(hr + F) + i);
-      for (int sp = 1; sp < a.splits; ++sp) {
-        const float* hs = hr + sp * a.out_split_stride;
-        const float4 gs = __ldcg(reinterpret_cast<const float4*>(hs) + i);
-        const float4 us = __ldcg(reinterpret_cast<const float4*>(hs + F) + i);
-        gv.x += gs.x; gv.y += gs.y; gv.z += gs.z; gv.w += gs.w;
-        uv.x += us.x; uv.y += us.y; uv.z += us.z; uv.w += us.w;
-      }
-      return make_float4(silu(gv.x) * uv.x, silu(gv.y) * uv.y, silu(gv.z) * uv.z,
-                         silu(gv.w) * uv.w);
-    };
-    float amax = 0.f;
-    for (int i = e; i < nv; i += 128) {
-      const float4 v = act4(i);
-      amax = fmaxf(fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y))), fmaxf(fabsf(v.z), fabsf(v.w)));
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    if (lane == 0) red[q] = amax;
-    named_bar_sync(1, 128);
-    const float am = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
-    if (e == 0) a.s2[r] = sc;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(a.aq + (size_t)r * F);
-    for (int i = e; i < nv; i += 128) {
-      const float4 v = act4(i);
-      dst[i] = static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.x, sc), __fdiv_rn(v.y, sc))) |
-               (static_cast<uint32_t>(e4m3x2(__fdiv_rn(v.z, sc), __fdiv_rn(v.w, sc))) << 16);
-    }
-    named_bar_sync(1, 128);                       // red[] is reused by the next row
-  }
-}
-
-// Channels 128 m .. 128 m + 127 of y for every token t < T: y = bf16_rne( sum_j w[t,j] *
-// (sum_s o[s][inv[t,j]]) + sum_s o[s][R + t] (shared expert) ), slots and splits in fixed order
-// -- the arithmetic of combine_kernel, so the result is bit-identical to it.
-__device__ __forceinline__ void fused_combine(const GemmArgs& a, int m, int R, int rows) {
-  const int e = threadIdx.x - 128, lane = threadIdx.x & 31, q = e >> 5;
-  const int d = a.out_ld;
-  const int ch = m * 128 + 4 * lane;
-  if (ch >= d) return;
-  for (int t = q; t < a.T; t += 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < a.k_max; ++j) {
-      const int r = a.inv_row[(size_t)t * a.k_max + j];
-      if (r < 0) continue;
-      if (r >= rows) {
-        report(a.status, kStatusDeviceCheck, kWhereCombine, t);
-        continue;
-      }
-      float4 v = __ldcg(reinterpret_cast<const float4*>(a.out + (size_t)r * d + ch));
-      for (int sp = 1; sp < a.splits; ++sp) {
-        const float4 u =
-            __ldcg(reinterpret_cast<const float4*>(a.out + sp * a.out_split_stride + (size_t)r * d + ch));
-        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
-      }
-      const float w = a.topk_w[(size_t)t * a.k_max + j];
-      acc.x = fmaf(w, v.x, acc.x);
-      acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z);
-      acc.w = fmaf(w, v.w, acc.w);
-    }
-    if (a.has_shared) {
-      for (int sp = 0; sp < a.splits; ++sp) {
-        const float4 u = __ldcg(reinterpret_cast<const float4*>(
-            a.out + sp * a.out_split_stride + (size_t)(R + t) * d + ch));
-        acc.x += u.x; acc.y += u.y; acc.z += u.z; acc.w += u.w;
-      }
-    }
-    const uint32_t lo = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.x))) |
-                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.y))) << 16);
-    const uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.z))) |
-                        (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.w))) << 16);
-    *reinterpret_cast<uint2*>(a.y + (size_t)t * d + ch) = make_uint2(lo, hi);
-    if (a.y_f32) *reinterpret_cast<float4*>(a.y_f32 + (size_t)t * d + ch) = acc;
-  }
-}
-
 template <int BN, int MODE, bool PAIR, int SLABS>
 __global__ void __launch_bounds__(256, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
@@ -259,9 +164,6 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);   // decode fusions
-  float* s_red = reinterpret_cast<float*>(tmem_slot + 2);                   // [4]
-  static_assert((2 * C::STAGES + 5) * 8 + 6 * 4 <= C::BAR_BYTES, "barrier area");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // A pair (2-CTA cluster) works on one tile of 256 x SLABS weight rows: CTA rank r holds the
@@ -329,47 +231,6 @@ __global__ void __launch_bounds__(256, 1)
     int stage = 0, issued = 0;
     uint32_t phase = 0;
     bool ok = true;
-    // L2 prefetch cursor (lane 0): the weight K-block kPrefetch blocks ahead of the next load, in
-    // this CTA's tile order. The loads then find their weights in L2, which deepens the pipeline
-    // beyond what shared memory holds (the weights come from HBM once either way).
-    constexpr int kPrefetch = C::STAGES;
-    int pf_tile = unit, pf_kb = -1, pf_kb1 = 0, pf_mc = 0, pf_ga = 0;
-    bool pf_sh = false, pf_end = false;
-    auto pf_step = [&]() {            // to the next weight K-block; false past the last tile
-      if (pf_end) return false;
-      if (pf_kb >= 0 && pf_kb + 1 < pf_kb1) {
-        ++pf_kb;
-        return true;
-      }
-      if (pf_kb >= 0) pf_tile += nunits;
-      if (pf_tile >= total_tiles) {
-        pf_end = true;
-        return false;
-      }
-      int pg, pmu, pn, ps;
-      decode_tile(tt, pf_tile, pg, pmu, pn, ps);
-      pf_mc = (PAIR ? 2 * pmu + static_cast<int>(crank) : pmu) * SLABS;
-      pf_sh = pg >= args.E_routed;
-      pf_ga = pf_sh ? 0 : pg;
-      pf_kb = ps * args.kb_per_split;
-      pf_kb1 = min(args.num_kb, pf_kb + args.kb_per_split);
-      return true;
-    };
-    auto pf_issue = [&]() {
-      const CUtensorMap* ma = pf_sh ? &map_a_shared : &map_a;
-#pragma unroll
-      for (int j = 0; j < SLABS; ++j) {
-        if (kGateUp) {
-          tma_prefetch_l2_4d(ma, pf_kb * kBK, (pf_mc + j) * 64, 0, pf_ga);
-          tma_prefetch_l2_4d(ma, pf_kb * kBK, (pf_mc + j) * 64, 1, pf_ga);
-        } else {
-          tma_prefetch_l2_3d(ma, pf_kb * kBK, (pf_mc + j) * 128, pf_ga);
-        }
-      }
-    };
-    if (lane == 0)
-      for (int i = 0; i < 2 * kPrefetch && pf_step(); ++i)
-        if (i >= kPrefetch) pf_issue();      // the first kPrefetch blocks are loaded right away
     for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
       int g, mu, n, s;
       decode_tile(tt, tile, g, mu, n, s);
@@ -459,7 +320,6 @@ __global__ void __launch_bounds__(256, 1)
             stage = 0;
             phase ^= 1u;
           }
-          if (pf_step()) pf_issue();
         }
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;   // lane 0's verdict for the whole warp
@@ -752,29 +612,6 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
       seq.advance(nh);
-      if constexpr (!PAIR && (MODE == kModeGateUpPartial || MODE == kModeDown)) {
-        // decode fusions: count this tile as finished (release: every epilogue thread's stores,
-        // then one counter update); the CTA that finishes the last tile of its token tile
-        // (gate/up) or of its output-channel tile (down) applies SwiGLU + requantisation or the
-        // weighted combine, then resets the counter
-        if (args.tile_done != nullptr) {
-          __threadfence();
-          named_bar_sync(1, 128);
-          const int cidx = MODE == kModeDown ? mc : tt.tp[g] + n;
-          const int total = MODE == kModeDown ? args.splits * tt.tp[tt.G] : tt.ms;
-          if (threadIdx.x == 128) *s_flag = atomicAdd(&args.tile_done[cidx], 1) == total - 1;
-          named_bar_sync(1, 128);
-          if (*s_flag) {
-            __threadfence();                          // acquire the other CTAs' outputs
-            if constexpr (MODE == kModeGateUpPartial)
-              fused_swiglu_requant(args, row0, nvalid, s_red);
-            else
-              fused_combine(args, mc, tt.off[args.E_routed], tt.off[tt.G]);
-            named_bar_sync(1, 128);
-            if (threadIdx.x == 128) args.tile_done[cidx] = 0;   // zero for the next call
-          }
-        }
-      }
     }
     if constexpr (C::DOWN_T) {
       if (lane == 0) bulk_wait_all();              // this warp's TMA stores have completed

@@ -28,13 +28,9 @@ struct Plan {
   int g1_kb, g1_m_tiles;                      // gate/up GEMM: K blocks (d/128), 64-row tiles
   int g1_splits, g1_kb_per_split;             // gate/up K split (decode); 1 = SwiGLU epilogue
   int g2_kb, g2_m_tiles, g2_splits, g2_kb_per_split;  // down GEMM
-  // decode tiles (BN <= 64): the gate/up GEMM always writes K-split partials and applies SwiGLU +
-  // requantisation itself (per token tile); fuse_combine: the down GEMM also combines (T <= 16)
-  bool fuse_swiglu, fuse_combine;
-  int n_tiles_cap;   // bound on the tile prefix: counters of the fused epilogues
   size_t off_status, off_part, off_ids, off_w, off_offsets, off_tiles, off_perm, off_inv, off_pscr;
   size_t off_xq, off_xs, off_xqp, off_xsp, off_amax, off_act, off_aq, off_s2, off_o, off_planes;
-  size_t off_hpart, off_counters;
+  size_t off_hpart;
   size_t bytes;
 };
 
@@ -66,23 +62,6 @@ struct GemmArgs {
   size_t out_split_stride;       // elements between split partials
   uint32_t* row_amax;            // gate/up: [Rpad] |act| max as fp32 bits
   int* status;
-  // Decode fusions (null counters = off). K-split gate/up: tile_done[tp[g] + n] counts the
-  // finished tiles of token tile n of group g; the CTA that finishes the last one applies SwiGLU
-  // and the FP8 requantisation to those rows (aq, s2 [Rpad], F = act width). Down: tile_done[m]
-  // counts the finished tiles of output-channel tile m; the CTA that finishes the last one
-  // computes the weighted combine of every token for those channels (y, y_f32 [T, d]; topk_w,
-  // inv_row [T, k_max]; the shared expert's rows follow the routed ones). Each last CTA resets
-  // its counter, so the counters stay zero between calls.
-  int* tile_done;
-  uint8_t* aq;
-  float* s2;
-  int F;
-  const float* topk_w;
-  const int32_t* inv_row;
-  int k_max;
-  int has_shared;
-  uint16_t* y;
-  float* y_f32;
 #ifdef MOE_WAIT_TEST
   int withhold;                  // wait-test build: skip the first tile's accumulator signal
 #endif
@@ -149,6 +128,8 @@ cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float
                               double* logits, int32_t* ids, float* w, uint8_t* xq, float* xs,
                               bool do_quant, int* status, const DecodeGrouping& grp,
                               cudaStream_t s);
+// Tokens per tile of the tensor-core router (64 or 128): the box height of map_x.
+int router_mma_tokens(int T, int E);
 // planes: 3 * E * d bf16 (workspace); map_w over planes [3][E][d], map_x over hidden [T][d]
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
                               const CUtensorMap& map_w, const CUtensorMap& map_x, double* logits,

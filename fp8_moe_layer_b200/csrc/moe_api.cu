@@ -134,10 +134,6 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
     p->g1_kb_per_split = (int)ceil_div(p->g1_kb, s1);
     p->g1_splits = (int)ceil_div(p->g1_kb, p->g1_kb_per_split);
   }
-  // decode tiles: SwiGLU + requantisation in the gate/up GEMM (one launch less), and for a handful
-  // of tokens the weighted combine in the down GEMM (one more)
-  p->fuse_swiglu = BN <= 64;
-  p->fuse_combine = BN <= 64 && T <= 16;
   const int m_rows2 = p->pair2 ? 256 : 128;      // weight rows of one down-GEMM work unit
   int s2 = choose_splits(est_ntiles * ceil_div(p->g2_m_tiles, m_rows2 / 128), p->g2_kb,
                          p->pair2 ? kPlanSMs / 2 : kPlanSMs, (double)m_rows2 * F,
@@ -147,11 +143,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
 
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + std::max<size_t>(bytes, 1)); return o; };
-  p->n_tiles_cap = (int)(ceil_div(p->Rcap, BN) + p->G + 2);
   p->off_status = take(256);
-  // counters of the fused decode epilogues, right after the status word: moe_forward clears both
-  // with one memset
-  p->off_counters = take(sizeof(int) * (size_t)std::max(p->n_tiles_cap, p->g2_m_tiles));
   p->off_part = take(sizeof(double) * (size_t)p->r_splits * T * E);
   p->off_ids = take(sizeof(int32_t) * (size_t)routed);
   p->off_w = take(sizeof(float) * (size_t)routed);
@@ -171,8 +163,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   p->off_s2 = take(sizeof(float) * (size_t)p->Rpad);
   p->off_o = take(sizeof(float) * (size_t)p->g2_splits * p->Rpad * d);
   p->off_planes = take(router_uses_mma(E, T, d) ? 3 * sizeof(uint16_t) * (size_t)E * d : 0);
-  p->off_hpart = take(p->g1_splits > 1 || p->fuse_swiglu
-                          ? sizeof(float) * p->g1_splits * (size_t)p->Rcap * 2 * F : 0);
+  p->off_hpart = take(p->g1_splits > 1 ? sizeof(float) * p->g1_splits * (size_t)p->Rcap * 2 * F : 0);
   p->bytes = off;
   return MOE_OK;
 }
@@ -234,11 +225,11 @@ static bool map_router_planes(CUtensorMap* m, const uint16_t* planes, int E, int
   const uint32_t box[3] = {64, 128, 1};
   return make_map(m, planes, 3, dims, str, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
-// bf16 hidden states [T][d]: box 64 (K) x 64 tokens.
-static bool map_hidden(CUtensorMap* m, const uint16_t* hidden, int T, int d) {
+// bf16 hidden states [T][d]: box 64 (K) x `tokens` tokens.
+static bool map_hidden(CUtensorMap* m, const uint16_t* hidden, int T, int d, int tokens) {
   const uint64_t dims[2] = {(uint64_t)d, (uint64_t)T};
   const uint64_t str[1] = {(uint64_t)d * 2};
-  const uint32_t box[2] = {64, 64};
+  const uint32_t box[2] = {64, (uint32_t)tokens};
   return make_map(m, hidden, 2, dims, str, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
@@ -293,7 +284,6 @@ struct Ws {
   float *w, *xs, *xsp, *act, *s2, *o, *hpart;
   uint16_t* planes;
   int32_t *ids, *offsets, *tiles, *perm, *inv, *pscr;
-  int* counters;
   uint8_t *xq, *xqp, *aq;
   uint32_t* amax;
 };
@@ -321,7 +311,6 @@ static Ws carve(const Plan& p, void* ws) {
   w.o = reinterpret_cast<float*>(b + p.off_o);
   w.planes = reinterpret_cast<uint16_t*>(b + p.off_planes);
   w.hpart = reinterpret_cast<float*>(b + p.off_hpart);
-  w.counters = reinterpret_cast<int*>(b + p.off_counters);
   return w;
 }
 
@@ -350,7 +339,8 @@ static int run_router_logits(const Plan& p, const Ws& w, const uint16_t* hidden,
                              const float* router_w, cudaStream_t s) {
   if (router_uses_mma(p)) {
     CUtensorMap mw, mx;
-    if (!map_router_planes(&mw, w.planes, p.E, p.d) || !map_hidden(&mx, hidden, p.T, p.d))
+    if (!map_router_planes(&mw, w.planes, p.E, p.d) ||
+        !map_hidden(&mx, hidden, p.T, p.d, router_mma_tokens(p.T, p.E)))
       return MOE_ERR_UNSUPPORTED;
     MOE_CUDA(launch_router_mma(p, router_w, w.planes, mw, mx, w.part, w.status, s));
     return MOE_OK;
@@ -361,23 +351,13 @@ static int run_router_logits(const Plan& p, const Ws& w, const uint16_t* hidden,
 
 // Grouped FFN: gate/up GEMM + SwiGLU, requantisation, down GEMM into `o` (split partials
 // `split_stride` apart).
-// Outputs of the weighted combine when the down GEMM computes it (decode fusion).
-struct CombineOut {
-  const float* topk_w;
-  const int32_t* inv_row;
-  uint16_t* y;
-  float* y_f32;
-};
-
-// Grouped FFN core shared by moe_forward and moe_grouped_ffn_fp8. `fuse` (moe_forward only)
-// allows the decode fusions of the plan; returns whether the down GEMM also combined into y.
+// Grouped FFN core shared by moe_forward and moe_grouped_ffn_fp8 (`gathered`: the grouping
+// kernel already laid the token rows out).
 static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* w13_scale,
                    const uint8_t* w2, const float* w2_scale, const uint8_t* w13s,
                    const float* w13s_scale, const uint8_t* w2s, const float* w2s_scale,
                    float* o, size_t split_stride, int64_t o_rows, void* const* ev,
-                   cudaStream_t s, const CombineOut* fuse, bool* combined,
-                   bool gathered = false) {
-  *combined = false;
+                   cudaStream_t s, bool gathered = false) {
   // gate/up B rows: decode tiles fetch token rows through the permutation (gather4), prefill
   // tiles read the gathered copy
   const bool gather4 = p.BN <= 64;
@@ -429,8 +409,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
 #ifdef MOE_WAIT_TEST
   g1.withhold = g_withhold_gemm_commit;
 #endif
-  const bool fuse_swiglu = fuse && p.fuse_swiglu;
-  const bool split1 = p.g1_splits > 1 || fuse_swiglu;
+  const bool split1 = p.g1_splits > 1;
   if (split1) {
     g1.splits = p.g1_splits;
     g1.kb_per_split = p.g1_kb_per_split;
@@ -439,19 +418,11 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
     g1.out_split_stride = (size_t)p.Rcap * 2 * p.F;
     g1.row_amax = nullptr;
   }
-  if (fuse_swiglu) {     // SwiGLU + requantisation by the CTA that finishes a token tile
-    g1.tile_done = w.counters;
-    g1.aq = w.aq;
-    g1.s2 = w.s2;
-    g1.F = p.F;
-  }
   record(4);
   MOE_CUDA(launch_gemm_gateup(p, m13, m13s, mx64, mx16, g1, split1, s));
 
   record(5);
-  if (fuse_swiglu) {
-    // (computed by the gate/up GEMM)
-  } else if (split1) {
+  if (split1) {
     MOE_CUDA(launch_swiglu_requant(p, w.hpart, p.g1_splits, g1.out_split_stride, total_rows, w.aq,
                                    w.s2, s));
   } else {
@@ -474,20 +445,9 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g2.out_ld = p.d;
   g2.out_split_stride = split_stride;
   g2.row_amax = nullptr;
-  g2.tile_done = nullptr;
 #ifdef MOE_WAIT_TEST
   g2.withhold = 0;
 #endif
-  if (fuse && p.fuse_combine) {   // the weighted combine by the CTA that finishes a channel tile
-    g2.tile_done = w.counters;
-    g2.topk_w = fuse->topk_w;
-    g2.inv_row = fuse->inv_row;
-    g2.k_max = p.k_max;
-    g2.has_shared = p.shared ? 1 : 0;
-    g2.y = fuse->y;
-    g2.y_f32 = fuse->y_f32;
-    *combined = true;
-  }
   // the down GEMM's TMA stores: o as [splits x split rows][d] fp32 (a caller's unsplit buffer
   // has exactly o_rows rows)
   CUtensorMap mo;
@@ -641,10 +601,8 @@ int moe_grouped_ffn_fp8(const moe_dims* dims, const uint16_t* hidden, const uint
   MOE_CUDA(cudaMemcpyAsync(w.perm, perm_token, sizeof(int32_t) * q.Rcap, cudaMemcpyDeviceToDevice, s));
   MOE_CUDA(cudaMemsetAsync(w.amax, 0, sizeof(uint32_t) * q.Rcap, s));   // the requant's row maxima
   const bool direct = p.g2_splits == 1;
-  bool combined = false;
   MOE_TRY(run_ffn(q, w, w13, w13_scale, w2, w2_scale, nullptr, nullptr, nullptr, nullptr,
-                  direct ? expert_out : w.o, (size_t)p.Rpad * p.d, q.Rcap, nullptr, s, nullptr,
-                  &combined));
+                  direct ? expert_out : w.o, (size_t)p.Rpad * p.d, q.Rcap, nullptr, s));
   if (!direct)
     MOE_CUDA(launch_reduce_splits(q, w.o, p.g2_splits, (size_t)p.Rpad * p.d, w.offsets + p.E,
                                   expert_out, s));
@@ -698,8 +656,7 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
     if (ev && ev[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
   };
 
-  // the status word and the counters of the fused decode epilogues
-  MOE_CUDA(cudaMemsetAsync(w.status, 0, p.off_counters + sizeof(int) * (size_t)std::max(p.n_tiles_cap, p.g2_m_tiles), s));
+  MOE_CUDA(cudaMemsetAsync(w.status, 0, 16, s));
   record(0);
   if (router_is_fused(p)) {
     // one kernel for stages 0 and 1 (stage 1's events bracket nothing)
@@ -735,15 +692,12 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
     gathered = true;
   }
   const size_t split_stride = (size_t)p.Rpad * p.d;
-  const CombineOut cout{w.w, w.inv, y, dbg ? dbg->y_f32 : nullptr};
-  bool combined = false;
   MOE_TRY(run_ffn(p, w, w13, w13_scale, w2, w2_scale, w13_shared, w13s_scale, w2_shared,
-                  w2s_scale, w.o, split_stride, p.Rcap, ev, s, &cout, &combined, gathered));
+                  w2s_scale, w.o, split_stride, p.Rcap, ev, s, gathered));
   record(7);
-  if (!combined)
-    MOE_CUDA(launch_combine(p, w.o, p.g2_splits, split_stride, w.w, w.inv,
-                            p.shared ? w.o : nullptr, p.shared ? w.offsets + p.E : nullptr,
-                            p.g2_splits, y, dbg ? dbg->y_f32 : nullptr, s));
+  MOE_CUDA(launch_combine(p, w.o, p.g2_splits, split_stride, w.w, w.inv,
+                          p.shared ? w.o : nullptr, p.shared ? w.offsets + p.E : nullptr,
+                          p.g2_splits, y, dbg ? dbg->y_f32 : nullptr, s));
   record(8);
   if (dbg) {
     const size_t kk = (size_t)p.T * p.k_max;

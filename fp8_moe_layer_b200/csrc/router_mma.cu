@@ -9,8 +9,10 @@
 // Method: "Routage MoE entre GPU" (viite.ai): the router scores every expert from the token's
 // hidden state. The top-k and the weights follow in topk_quant_kernel (route.cu).
 //
-// Tiles: 128 experts (MMA M, TMEM lanes) x 64 tokens (MMA N); K-step = 64 bf16 = one 128-byte
-// swizzled row. One stage holds the three weight planes and the token tile (56 KB), four stages.
+// Tiles: 128 experts (MMA M, TMEM lanes) x NT tokens (MMA N, 64 or 128); K-step = 64 bf16 = one
+// 128-byte swizzled row. One stage holds the three weight planes and the token tile (56 or 64 KB;
+// four or three stages). 128-token tiles halve the weight bytes per MMA; they are used when they
+// still give about a wave of tiles (DeepSeek-V3 T=8192: 128 tiles instead of 1.7 waves of 64).
 // Persistent grid, one CTA per SM, warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = TMEM
 // allocator, warps 4-7 = epilogue (fp32 logits, coalesced over experts). Bounded waits as in
 // gemm.cu.
@@ -19,12 +21,14 @@
 
 namespace moe {
 
-constexpr int kRtN = 64;                         // tokens per tile
 constexpr int kRtPlaneBytes = 128 * kBK;         // 128 experts x 64 bf16
-constexpr int kRtBBytes = kRtN * kBK;            // 64 tokens x 64 bf16
-constexpr int kRtStageBytes = 3 * kRtPlaneBytes + kRtBBytes;
-constexpr int kRtStages = 4;
-constexpr int kRtSmem = 1024 + kRtStages * kRtStageBytes + 256;
+template <int NT>
+struct RtCfg {
+  static constexpr int B_BYTES = NT * kBK;                       // NT tokens x 64 bf16
+  static constexpr int STAGE_BYTES = 3 * kRtPlaneBytes + B_BYTES;
+  static constexpr int STAGES = NT == 64 ? 4 : 3;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+};
 
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
@@ -59,11 +63,14 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
   }
 }
 
+template <int kRtN>
 __global__ void __launch_bounds__(256, 1)
     router_mma_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
                       int T, int E, int num_kb, double* __restrict__ logits, int* status) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
+  constexpr int kRtStageBytes = RtCfg<kRtN>::STAGE_BYTES;
+  constexpr int kRtStages = RtCfg<kRtN>::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRtStages * kRtStageBytes);
@@ -218,6 +225,31 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+int router_mma_tokens(int T, int E) {
+  return ((E + 127) / 128) * ((T + 127) / 128) >= 100 ? 128 : 64;
+}
+
+template <int NT>
+static cudaError_t launch_router_mma_t(const Plan& p, const CUtensorMap& map_w,
+                                       const CUtensorMap& map_x, double* logits, int* status,
+                                       cudaStream_t s) {
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 64 && !attr_done[dev]) {
+    err = cudaFuncSetAttribute(router_mma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               RtCfg<NT>::SMEM);
+    if (err != cudaSuccess) return err;
+    attr_done[dev] = true;
+  }
+  const int tiles = ((p.E + 127) / 128) * ((p.T + NT - 1) / NT);
+  const int grid = std::min(tiles, num_sms());
+  launch_pdl(router_mma_kernel<NT>, dim3(grid), dim3(256), RtCfg<NT>::SMEM, s, map_w, map_x, p.T,
+             p.E, (p.d + 63) / 64, logits, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
                               const CUtensorMap& map_w, const CUtensorMap& map_x, double* logits,
                               int* status, cudaStream_t s) {
@@ -226,20 +258,9 @@ cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* pl
   launch_pdl(router_split_kernel, dim3(split_blocks), dim3(256), 0, s, router_w, n, planes);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-  if (dev < 64 && !attr_done[dev]) {
-    err = cudaFuncSetAttribute(router_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kRtSmem);
-    if (err != cudaSuccess) return err;
-    attr_done[dev] = true;
-  }
-  const int tiles = ((p.E + 127) / 128) * ((p.T + kRtN - 1) / kRtN);
-  const int grid = std::min(tiles, num_sms());
-  launch_pdl(router_mma_kernel, dim3(grid), dim3(256), kRtSmem, s, map_w, map_x, p.T, p.E, (p.d + 63) / 64, logits,
-                                               status);
-  return cudaGetLastError();
+  return router_mma_tokens(p.T, p.E) == 128
+             ? launch_router_mma_t<128>(p, map_w, map_x, logits, status, s)
+             : launch_router_mma_t<64>(p, map_w, map_x, logits, status, s);
 }
 
 }  // namespace moe
