@@ -220,29 +220,6 @@ __device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// Four rows of a 2-D tensor whose map has a one-row box of 128 bytes (tile::gather4): rows r0..r3
-// at column x land in four consecutive 128-byte rows of shared memory at dst (swizzled like a
-// 4-row tile load). The pair form counts the bytes on the barrier at `bar` (shared::cluster).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
-                                            int r0, int r1, int r2, int r3, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2),
-      "r"(r3), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map, uint32_t bar,
-                                                 int x, int r0, int r1, int r2, int r3,
-                                                 uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
-      ".mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;"
-      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0),
-      "r"(r1), "r"(r2), "r"(r3), "l"(policy)
-      : "memory");
-}
-
 // TMA tensor store from shared memory (bulk async-group completion), and the group waits.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
   asm volatile(

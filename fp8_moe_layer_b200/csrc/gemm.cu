@@ -49,15 +49,10 @@ struct GemmCfg {
   static constexpr int SMEM_MAX = 232448;                  // 227 KB per block
   // group offsets and tile prefix of up to kMaxExperts + 1 groups, cached in shared memory
   static constexpr int TABLE_BYTES = 2 * (kMaxExperts + 2) * 4;
-  // gate/up with decode tiles: the tokens of the tile's rows this CTA loads (indices for the
-  // gather4 loads); prefill tiles load rows of a gathered copy with 64- and 16-row boxes
-  static constexpr bool GATHER = MODE != kModeDown && BN <= 64;
-  static constexpr int ROWIDX_BYTES = GATHER ? BROWS * 4 : 0;
   static constexpr int STAGES_FIT =
-      (SMEM_MAX - 1024 - XCHG_BYTES - BAR_BYTES - TABLE_BYTES - ROWIDX_BYTES) / STAGE_BYTES;
+      (SMEM_MAX - 1024 - XCHG_BYTES - BAR_BYTES - TABLE_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-  static constexpr int SMEM =
-      1024 + STAGES * STAGE_BYTES + XCHG_BYTES + BAR_BYTES + TABLE_BYTES + ROWIDX_BYTES;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + XCHG_BYTES + BAR_BYTES + TABLE_BYTES;
   // TMEM: two halves, each holding one tile's accumulators (double buffering). One slab: a half
   // is BN columns. Two slabs: a half is 256 columns; a tile of <= 128 valid token columns keeps
   // both slabs' accumulators in one half (slab j at column 128 j), a wider tile takes both
@@ -180,7 +175,6 @@ __global__ void __launch_bounds__(256, 1)
   if (unit >= total_tiles) return;
   int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
   int* s_tp = s_off + (kMaxExperts + 2);
-  int* s_rows = s_tp + (kMaxExperts + 2);           // [BROWS] gather4 row indices (gate/up)
   for (int i = threadIdx.x; i <= args.G; i += blockDim.x) {
     s_off[i] = args.group_offsets[i];
     s_tp[i] = args.tile_prefix[i];
@@ -218,40 +212,25 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tempty_l = PAIR ? cluster_addr(tempty, 0) : 0u;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (lane 0 issues;
-    // for the gate/up GEMM the whole warp first stages the tokens of the tile's rows)
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_map(&map_a);
       tma_prefetch_map(&map_a_shared);
       tma_prefetch_map(&map_b64);
       tma_prefetch_map(&map_b16);
-    }
-    const uint64_t pol_w = l2_policy_evict_first();   // weights: streamed once
-    const uint64_t pol_x = l2_policy_evict_last();    // activations: reused by every m-tile
-    int stage = 0, issued = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
-      int g, mu, n, s;
-      decode_tile(tt, tile, g, mu, n, s);
-      const int mc = (PAIR ? 2 * mu + static_cast<int>(crank) : mu) * SLABS;  // first m-tile
-      const int row0 = tt.off[g] + n * BN;
-      const int rowsN = tile_rows_rounded<BN, C::ROUND>(tt, g, row0);   // the MMA's N
-      const int myrows = PAIR ? rowsN / 2 : rowsN;       // token rows this CTA loads
-      const int myrow0 = row0 + static_cast<int>(crank) * myrows;
-      if constexpr (C::GATHER) {
-        // tokens of this CTA's rows; rows past the group's end (the MMA's N is rounded up) and
-        // tokens outside [0, T) (caller-provided permutation) fetch row 0, whose columns the
-        // epilogue ignores or scales by 0
-        const int gend = tt.off[g + 1];
-        for (int i = lane; i < myrows; i += 32) {
-          const int r = myrow0 + i;
-          int t = r < gend ? args.row_token[r] : 0;
-          s_rows[i] = (t >= 0 && t < args.T) ? t : 0;
-        }
-        __syncwarp();
-      }
-      if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();   // weights: streamed once
+      const uint64_t pol_x = l2_policy_evict_last();    // activations: reused by every m-tile
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = unit; ok && tile < total_tiles; tile += nunits) {
+        int g, mu, n, s;
+        decode_tile(tt, tile, g, mu, n, s);
+        const int mc = (PAIR ? 2 * mu + static_cast<int>(crank) : mu) * SLABS;  // first m-tile
+        const int row0 = tt.off[g] + n * BN;
+        const int rowsN = tile_rows_rounded<BN, C::ROUND>(tt, g, row0);   // the MMA's N
+        const int myrows = PAIR ? rowsN / 2 : rowsN;       // token rows this CTA loads
+        const int myrow0 = row0 + static_cast<int>(crank) * myrows;
         // bytes that complete the (even CTA's) full barrier: both CTAs' loads for a pair
         const uint32_t stage_bytes = (PAIR ? 2 : 1) * C::A_BYTES + rowsN * kBK;
         const int kb0 = s * args.kb_per_split;
@@ -283,17 +262,11 @@ __global__ void __launch_bounds__(256, 1)
                 tma_load_3d_pair(sj, ma, fb, kb * kBK, (mc + j) * 128, ga, pol_w);
               }
             }
-            if constexpr (C::GATHER) {
-              for (int r = 0; r < myrows; r += 4)
-                tma_gather4_pair(sb + r * kBK, &map_b64, fb, kb * kBK, s_rows[r], s_rows[r + 1],
-                                 s_rows[r + 2], s_rows[r + 3], pol_x);
-            } else {
-              int r = 0;
-              for (; r + 64 <= myrows; r += 64)
-                tma_load_2d_pair(sb + r * kBK, &map_b64, fb, kb * kBK, myrow0 + r, pol_x);
-              for (; r < myrows; r += 16)
-                tma_load_2d_pair(sb + r * kBK, &map_b16, fb, kb * kBK, myrow0 + r, pol_x);
-            }
+            int r = 0;
+            for (; r + 64 <= myrows; r += 64)
+              tma_load_2d_pair(sb + r * kBK, &map_b64, fb, kb * kBK, myrow0 + r, pol_x);
+            for (; r < myrows; r += 16)
+              tma_load_2d_pair(sb + r * kBK, &map_b16, fb, kb * kBK, myrow0 + r, pol_x);
           } else {
             if (kGateUp) {
               tma_load_4d(sa, ma, &full[stage], kb * kBK, mc * 64, 0, ga, pol_w);
@@ -301,19 +274,13 @@ __global__ void __launch_bounds__(256, 1)
             } else {
               tma_load_3d(sa, ma, &full[stage], kb * kBK, mc * 128, ga, pol_w);
             }
-            if constexpr (C::GATHER) {
-              for (int r = 0; r < myrows; r += 4)
-                tma_gather4(sb + r * kBK, &map_b64, &full[stage], kb * kBK, s_rows[r],
-                            s_rows[r + 1], s_rows[r + 2], s_rows[r + 3], pol_x);
-            } else {
-              // only the tile's valid token rows: 64-row boxes, then 16-row boxes
-              int r = 0;
-              if constexpr (BN >= 64)
-                for (; r + 64 <= myrows; r += 64)
-                  tma_load_2d(sb + r * kBK, &map_b64, &full[stage], kb * kBK, myrow0 + r, pol_x);
-              for (; r < myrows; r += 16)
-                tma_load_2d(sb + r * kBK, &map_b16, &full[stage], kb * kBK, myrow0 + r, pol_x);
-            }
+            // only the tile's valid token rows: 64-row boxes, then 16-row boxes
+            int r = 0;
+            if constexpr (BN >= 64)
+              for (; r + 64 <= myrows; r += 64)
+                tma_load_2d(sb + r * kBK, &map_b64, &full[stage], kb * kBK, myrow0 + r, pol_x);
+            for (; r < myrows; r += 16)
+              tma_load_2d(sb + r * kBK, &map_b16, &full[stage], kb * kBK, myrow0 + r, pol_x);
           }
           ++issued;
           if (++stage == C::STAGES) {
@@ -322,13 +289,9 @@ __global__ void __launch_bounds__(256, 1)
           }
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;   // lane 0's verdict for the whole warp
-      __syncwarp();                                     // s_rows may be overwritten now
-    }
-    // Drain: the most recent load of every stage must have landed before the CTA exits. (In a
-    // pair the even CTA's full barriers count both CTAs' bytes; the odd CTA relies on the final
-    // cluster barrier, which the even CTA reaches only after this drain.)
-    if (lane == 0) {
+      // Drain: the most recent load of every stage must have landed before the CTA exits. (In
+      // a pair the even CTA's full barriers count both CTAs' bytes; the odd CTA relies on the
+      // final cluster barrier, which the even CTA reaches only after this drain.)
       const int outstanding = leader ? min(issued, C::STAGES) : 0;
       for (int i = 0; i < outstanding; ++i) {
         int st = stage - 1 - i;
@@ -452,17 +415,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int u = 0; u < kRsRegs; ++u) {
         const int c = u * C::CW + lane;
-        float v = 0.f;
-        if (c < nvalid && (C::CW == 32 || lane < C::CW)) {
-          if constexpr (C::GATHER) {
-            const int t = args.row_token[row0 + c];
-            if (t >= 0 && t < args.T) v = args.token_scale[t];
-            else report(args.status, kStatusDeviceCheck, kWhere, row0 + c);
-          } else {
-            v = args.row_scale[row0 + c];
-          }
-        }
-        rs[u] = v;
+        rs[u] = (c < nvalid && (C::CW == 32 || lane < C::CW)) ? args.row_scale[row0 + c] : 0.f;
       }
       const bool sh = g >= args.E_routed;
       const float* wsc = sh ? args.w_scale_shared : args.w_scale + (size_t)g * args.w_scale_ld;

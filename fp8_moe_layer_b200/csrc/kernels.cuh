@@ -47,13 +47,7 @@ struct GemmArgs {
   int G, E_routed;               // groups >= E_routed use the shared-expert weights
   int m_tiles, splits, kb_per_split, num_kb;
   int M_valid;                   // valid weight rows: F (gate/up halves) or d (down)
-  const float* row_scale;        // down: [Rpad] activation scale of each routed row
-  // gate/up with decode tiles (BN <= 64): token rows fetched through the permutation
-  // (tile::gather4 loads from the quantised hidden states [T, d]); the scale of routed row r is
-  // token_scale[row_token[r]] instead of row_scale[r]
-  const int32_t* row_token;      // [Rpad] token of each routed row
-  const float* token_scale;      // [T]
-  int T;
+  const float* row_scale;        // [Rpad] activation scale of each routed row
   const float* w_scale;          // [E, w_scale_ld] per-output-channel weight scales
   const float* w_scale_shared;   // [w_scale_ld] shared expert (or null)
   int w_scale_ld;                // 2F (gate/up) or d (down)
@@ -155,9 +149,7 @@ cudaError_t launch_tile_prefix(const Plan& p, const int32_t* offsets, int32_t* t
 cudaError_t launch_gather(const Plan& p, const uint8_t* xq, const float* xs, const int32_t* perm,
                           const int32_t* total_rows, uint8_t* xqp, float* xsp, uint32_t* amax,
                           int* status, cudaStream_t s);
-// acts64 / acts16: the B rows' maps -- the routed-row activations with 64-row and 16-row TMA
-// boxes, or (gate/up with decode tiles) the quantised hidden states with one-row boxes for
-// tile::gather4 (acts16 then unused)
+// acts64 / acts16: the routed-row activations with 64-row and 16-row TMA boxes
 cudaError_t launch_gemm_gateup(const Plan& p, const CUtensorMap& w13, const CUtensorMap& w13s,
                                const CUtensorMap& acts64, const CUtensorMap& acts16,
                                const GemmArgs& a, bool partial, cudaStream_t s);

@@ -154,9 +154,8 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   p->off_pscr = take(sizeof(int32_t) * 2 * (size_t)permute_blocks(*p) * E);
   p->off_xq = take((size_t)T * d);
   p->off_xs = take(sizeof(float) * (size_t)T);
-  // permuted copy of the quantised token rows: prefill-sized tiles only (decode tiles gather)
-  p->off_xqp = take(BN >= 128 ? (size_t)p->Rpad * d : 0);
-  p->off_xsp = take(BN >= 128 ? sizeof(float) * (size_t)p->Rpad : 0);
+  p->off_xqp = take((size_t)p->Rpad * d);
+  p->off_xsp = take(sizeof(float) * (size_t)p->Rpad);
   p->off_amax = take(sizeof(uint32_t) * (size_t)p->Rpad);
   p->off_act = take(sizeof(float) * (size_t)p->Rpad * F);
   p->off_aq = take((size_t)p->Rpad * F);
@@ -246,13 +245,6 @@ static bool map_w2(CUtensorMap* m, const uint8_t* w, int experts, int d, int F) 
   const uint64_t str[2] = {(uint64_t)F, (uint64_t)d * F};
   const uint32_t box[3] = {(uint32_t)kBK, 128, 1};
   return make_map(m, w, 3, dims, str, box);
-}
-// Quantised hidden states [T, d] for tile::gather4 loads: box 128 (K) x 1 row.
-static bool map_token_rows(CUtensorMap* m, const uint8_t* xq, int T, int d) {
-  const uint64_t dims[2] = {(uint64_t)d, (uint64_t)std::max(T, 1)};
-  const uint64_t str[1] = {(uint64_t)d};
-  const uint32_t box[2] = {(uint32_t)kBK, 1};
-  return make_map(m, xq, 2, dims, str, box);
 }
 // Row-major activations [rows, K]: box 128 (K) x BN rows.
 static bool map_rows(CUtensorMap* m, const uint8_t* a, int64_t rows, int K, int BN) {
@@ -358,15 +350,9 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
                    const float* w13s_scale, const uint8_t* w2s, const float* w2s_scale,
                    float* o, size_t split_stride, int64_t o_rows, void* const* ev,
                    cudaStream_t s, bool gathered = false) {
-  // gate/up B rows: decode tiles fetch token rows through the permutation (gather4), prefill
-  // tiles read the gathered copy
-  const bool gather4 = p.BN <= 64;
   CUtensorMap m13, m13s, mx64, mx16, m2, m2s, maq64, maq16;
-  const bool maps_x = gather4 ? map_token_rows(&mx64, w.xq, p.T, p.d) &&
-                                    map_token_rows(&mx16, w.xq, p.T, p.d)
-                              : map_rows(&mx64, w.xqp, p.Rpad, p.d, 64) &&
-                                    map_rows(&mx16, w.xqp, p.Rpad, p.d, 16);
-  if (!map_w13(&m13, w13, p.E, p.F, p.d) || !map_w2(&m2, w2, p.E, p.d, p.F) || !maps_x ||
+  if (!map_w13(&m13, w13, p.E, p.F, p.d) || !map_w2(&m2, w2, p.E, p.d, p.F) ||
+      !map_rows(&mx64, w.xqp, p.Rpad, p.d, 64) || !map_rows(&mx16, w.xqp, p.Rpad, p.d, 16) ||
       !map_rows(&maq64, w.aq, p.Rpad, p.F, 64) || !map_rows(&maq16, w.aq, p.Rpad, p.F, 16))
     return MOE_ERR_UNSUPPORTED;
   m13s = m13;
@@ -381,7 +367,7 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   const int32_t* total_rows = w.offsets + p.G;     // offsets[G] = routed (+ shared) rows
 
   record(3);
-  if (!gather4 && !gathered)   // (else the grouping kernel already laid the rows out)
+  if (!gathered)   // (else the grouping kernel already laid the rows out)
     MOE_CUDA(launch_gather(p, w.xq, w.xs, w.perm, total_rows, w.xqp, w.xsp, w.amax, w.status, s));
 
   GemmArgs g1{};
@@ -395,9 +381,6 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g1.num_kb = p.g1_kb;
   g1.M_valid = p.F;
   g1.row_scale = w.xsp;
-  g1.row_token = w.perm;
-  g1.token_scale = w.xs;
-  g1.T = p.T;
   g1.w_scale = w13_scale;
   g1.w_scale_shared = w13s_scale;
   g1.w_scale_ld = 2 * p.F;
@@ -436,8 +419,6 @@ static int run_ffn(const Plan& p, const Ws& w, const uint8_t* w13, const float* 
   g2.num_kb = p.g2_kb;
   g2.M_valid = p.d;
   g2.row_scale = w.s2;
-  g2.row_token = nullptr;
-  g2.token_scale = nullptr;
   g2.w_scale = w2_scale;
   g2.w_scale_shared = w2s_scale;
   g2.w_scale_ld = p.d;
@@ -599,7 +580,6 @@ int moe_grouped_ffn_fp8(const moe_dims* dims, const uint16_t* hidden, const uint
   MOE_CUDA(cudaMemcpyAsync(w.offsets, expert_offsets, sizeof(int32_t) * (p.E + 1),
                            cudaMemcpyDeviceToDevice, s));
   MOE_CUDA(cudaMemcpyAsync(w.perm, perm_token, sizeof(int32_t) * q.Rcap, cudaMemcpyDeviceToDevice, s));
-  MOE_CUDA(cudaMemsetAsync(w.amax, 0, sizeof(uint32_t) * q.Rcap, s));   // the requant's row maxima
   const bool direct = p.g2_splits == 1;
   MOE_TRY(run_ffn(q, w, w13, w13_scale, w2, w2_scale, nullptr, nullptr, nullptr, nullptr,
                   direct ? expert_out : w.o, (size_t)p.Rpad * p.d, q.Rcap, nullptr, s));
@@ -678,12 +658,11 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                                w.status, s));
   }
   record(2);
-  // grouping: by the decode router itself (T <= 8), alone (decode tiles: the gate/up GEMM fetches
-  // the rows), with the row gather in one kernel (prefill tiles, T * k_max <= 8192), or followed
-  // by the gather kernel
+  // grouping: by the decode router itself (T <= 8), with the row gather in one kernel
+  // (T * k_max <= 8192), or alone; the gather kernel follows in the last two cases
   bool gathered = false;
   if (router_uses_gemv(p)) {
-  } else if (p.BN <= 64 || !permute_gather_fused(p)) {
+  } else if (!permute_gather_fused(p)) {
     MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
                             w.status, s));
   } else {

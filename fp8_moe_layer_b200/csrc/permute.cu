@@ -1,10 +1,10 @@
 // Grouping of the routed (token, slot) pairs by expert: per-warp histograms, an exclusive prefix
-// sum over experts, and a stable scatter so routed rows are ordered by (expert, token). Then, for
-// prefill-sized token tiles, the gather that lays the quantised token rows out in that order for
-// the grouped GEMMs. (Decode-sized tiles skip it: their gate/up GEMM fetches the few rows of a tile
-// through the permutation with tile::gather4 loads. At prefill those four-row loads -- 32 per
-// pipeline stage of a 256-token tile -- made the GEMM TMA-issue-bound: 7650 vs 2659 us at
-// DeepSeek T=8192, so a gathered copy it is.)
+// sum over experts, and a stable scatter so routed rows are ordered by (expert, token). Then the
+// gather that lays the quantised token rows out in that order for the grouped GEMMs. (The GEMM
+// could fetch the rows through the permutation with four-row tile::gather4 TMA loads instead;
+// measured on B200 that is slower at every batch size -- the 32 gather4 loads per pipeline stage
+// of a 256-token tile make the gate/up GEMM TMA-issue-bound, 7650 vs 2659 us at DeepSeek T=8192,
+// and decode layers lose 0.4-230 us -- so the rows are gathered.)
 //
 // Method: "Routage MoE entre GPU" (viite.ai) -- only the selected experts process a token; the
 // tokens are dispatched to their experts and their order restored at the combine.
