@@ -17,7 +17,10 @@ LIB = os.path.join(HERE, "libfp8moe.so")
 # switch that withholds one GEMM signal (include/moe_testing.h), for the tests of the
 # device-timeout path. Nothing but those tests loads it.
 LIB_WAITTEST = os.path.join(HERE, "libfp8moe_waittest.so")
-VARIANTS = {LIB: [], LIB_WAITTEST: ["-DMOE_WAIT_TEST"]}
+# The role-counter build: the grouped GEMMs add up the cycles each warp role waits
+# (include/moe_testing.h; fp8_moe_layer_b200/role_counters.py reads them).
+LIB_ROLES = os.path.join(HERE, "libfp8moe_roles.so")
+VARIANTS = {LIB: [], LIB_WAITTEST: ["-DMOE_WAIT_TEST"], LIB_ROLES: ["-DMOE_ROLE_COUNTERS"]}
 SOURCES = ["moe_api.cu", "route.cu", "router_mma.cu", "permute.cu", "gemm.cu", "combine.cu",
            "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -67,7 +70,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
 
 
 if __name__ == "__main__":
-    for target in ([LIB, LIB_WAITTEST] if "--all" in sys.argv else [LIB]):
+    for target in ([LIB, LIB_WAITTEST, LIB_ROLES] if "--all" in sys.argv else [LIB]):
         build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv,
               lib=target)
         print(target)

@@ -32,6 +32,21 @@
 
 namespace moe {
 
+#ifdef MOE_ROLE_COUNTERS
+// Role-counter build only: cycles each warp role of each CTA spent waiting, per GEMM mode
+// ([mode][cta][counter]): 0 producer waiting for a free stage, 1 MMA issuer waiting for a free
+// accumulator, 2 MMA issuer waiting for a stage's data, 3 K blocks issued, 4 epilogue waiting for
+// an accumulator, 5 cycles from set-up to the end, 6 tiles.
+constexpr int kRoleMaxCtas = 256;
+__device__ unsigned long long g_role_cycles[3][kRoleMaxCtas][8];
+#define MOE_ROLE_T0(v) const unsigned long long v = clock64()
+#define MOE_ROLE_ADD(mode, i, val) \
+  do { if (blockIdx.x < kRoleMaxCtas) g_role_cycles[mode][blockIdx.x][i] += (val); } while (0)
+#else
+#define MOE_ROLE_T0(v)
+#define MOE_ROLE_ADD(mode, i, val)
+#endif
+
 template <int BN, int MODE, bool PAIR, int SLABS = 1>
 struct GemmCfg {
   static constexpr int BM = 128;                           // weight rows of one slab
@@ -207,6 +222,7 @@ __global__ void __launch_bounds__(256, 1)
   else __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  MOE_ROLE_T0(t_setup);
   // shared::cluster addresses of the even CTA's barriers (pair loads, commits and arrivals)
   const uint32_t full_l = PAIR ? cluster_addr(full, 0) : 0u;
   const uint32_t tempty_l = PAIR ? cluster_addr(tempty, 0) : 0u;
@@ -239,8 +255,10 @@ __global__ void __launch_bounds__(256, 1)
         const CUtensorMap* ma = sh ? &map_a_shared : &map_a;
         const int ga = sh ? 0 : g;
         for (int kb = kb0; kb < kb1; ++kb) {
+          MOE_ROLE_T0(tq0);
           const bool got = PAIR ? mbar_wait_cluster(&empty[stage], phase ^ 1u)
                                 : mbar_wait(&empty[stage], phase ^ 1u);
+          MOE_ROLE_ADD(MODE, 0, clock64() - tq0);
           if (!got) {
             report(args.status, kStatusDeviceTimeout, kWhere, 1);
             ok = false;
@@ -328,8 +346,10 @@ __global__ void __launch_bounds__(256, 1)
         uint32_t ph[2], col[SLABS];
         const int nh = seq.take(ncols, h, ph, col);
         for (int i = 0; ok && i < nh; ++i) {
+          MOE_ROLE_T0(tq0);
           const bool freed = PAIR ? mbar_wait_cluster(&tempty[h[i]], ph[i] ^ 1u)
                                   : mbar_wait(&tempty[h[i]], ph[i] ^ 1u);
+          MOE_ROLE_ADD(MODE, 1, clock64() - tq0);
           if (!freed) {
             report(args.status, kStatusDeviceTimeout, kWhere, 2);
             ok = false;
@@ -338,7 +358,11 @@ __global__ void __launch_bounds__(256, 1)
         if (!ok) break;
         tc_fence_after_sync();
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase)) {
+          MOE_ROLE_T0(tf0);
+          const bool landed = mbar_wait(&full[stage], phase);
+          MOE_ROLE_ADD(MODE, 2, clock64() - tf0);
+          MOE_ROLE_ADD(MODE, 3, 1ull);
+          if (!landed) {
             report(args.status, kStatusDeviceTimeout, kWhere, 3);
             ok = false;
             break;
@@ -438,8 +462,10 @@ __global__ void __launch_bounds__(256, 1)
           wsv = valid ? wsc[ch] : 0.f;
         }
         if (!bad && (j == 0 || nh == 2)) {
+          MOE_ROLE_T0(te0);
           const bool ok = PAIR ? mbar_wait_cluster(&tfull[h[hi]], ph[hi])
                                : mbar_wait(&tfull[h[hi]], ph[hi]);
+          if (warp == 4 && lane == 0) MOE_ROLE_ADD(MODE, 4, clock64() - te0);
           bad = __any_sync(0xffffffffu, !ok);       // warp-uniform: TMEM loads are .sync.aligned
           if (bad && lane == 0) report(args.status, kStatusDeviceTimeout, kWhere, 5);
         }
@@ -571,6 +597,10 @@ __global__ void __launch_bounds__(256, 1)
     }
   }
 
+  if (warp == 4 && lane == 0) {
+    MOE_ROLE_ADD(MODE, 5, clock64() - t_setup);
+    MOE_ROLE_ADD(MODE, 6, (unsigned long long)((total_tiles - unit + nunits - 1) / nunits));
+  }
   tc_fence_before_sync();
   if constexpr (PAIR) cluster_sync_all();   // no CTA leaves while its pair still uses its memory
   else __syncthreads();
@@ -679,3 +709,14 @@ cudaError_t launch_gemm_down(const Plan& p, const CUtensorMap& w2, const CUtenso
 }
 
 }  // namespace moe
+
+#ifdef MOE_ROLE_COUNTERS
+extern "C" int moe_role_counters_read(uint64_t* out) {
+  return cudaMemcpyFromSymbol(out, moe::g_role_cycles, sizeof(moe::g_role_cycles)) == cudaSuccess
+             ? 0 : -4;
+}
+extern "C" int moe_role_counters_reset(void) {
+  static unsigned long long zero[3 * moe::kRoleMaxCtas * 8] = {};
+  return cudaMemcpyToSymbol(moe::g_role_cycles, zero, sizeof(zero)) == cudaSuccess ? 0 : -4;
+}
+#endif

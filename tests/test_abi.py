@@ -139,17 +139,22 @@ def test_binding_argument_counts_match_the_header(ops):
         assert len(fn.argtypes) == _nargs(sig), name
 
 
-def test_wait_test_build_exports_its_switch_and_the_library_does_not():
+def test_test_builds_export_their_entry_points_and_the_library_does_not():
     from fp8_moe_layer_b200 import build
     path = build.build(lib=build.LIB_WAITTEST)
     text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "moe_testing.h")).read(),
                   flags=re.S)
     names = sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
-    assert names == ["moe_test_withhold_gemm_commit"]
+    assert names == ["moe_role_counters_read", "moe_role_counters_reset",
+                     "moe_test_withhold_gemm_commit"]
     test_lib = ctypes.CDLL(path)
+    roles_lib = ctypes.CDLL(build.build(lib=build.LIB_ROLES))
     prod = ctypes.CDLL(os.path.join(ROOT, "fp8_moe_layer_b200", "libfp8moe.so"))
+    assert hasattr(test_lib, "moe_test_withhold_gemm_commit")
+    assert hasattr(roles_lib, "moe_role_counters_read")
+    assert hasattr(roles_lib, "moe_role_counters_reset")
     for n in names:
-        assert hasattr(test_lib, n)
         assert not hasattr(prod, n)
     for n in declared_functions():
         assert hasattr(test_lib, n), n
+        assert hasattr(roles_lib, n), n
