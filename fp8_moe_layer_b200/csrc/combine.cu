@@ -97,8 +97,23 @@ __global__ void __launch_bounds__(1024) swiglu_requant_kernel(
   }
 }
 
+// Eight consecutive fp32 values of row r (K-split partials summed in split order).
+__device__ __forceinline__ void load8_rows(const float* o, int splits, size_t split_stride,
+                                           int64_t r, int d, int i, float (&v)[8]) {
+  const float4* p = reinterpret_cast<const float4*>(o + (size_t)r * d) + 2 * i;
+  float4 a = p[0], b = p[1];
+  for (int s = 1; s < splits; ++s) {
+    const float4* q = reinterpret_cast<const float4*>(o + s * split_stride + (size_t)r * d) + 2 * i;
+    const float4 c = q[0], e = q[1];
+    a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
+    b.x += e.x; b.y += e.y; b.z += e.z; b.w += e.w;
+  }
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
 // y[t, :] = bf16_rne( sum_j w[t, j] * (sum_s o[s][inv[t, j], :]) + sum_s shared[s][row0 + t, :] )
-// Slots with inv < 0 are skipped; fp32, slot order and split order fixed (deterministic).
+// Slots with inv < 0 are skipped; fp32, slot order and split order fixed (deterministic). A
+// thread takes 8 channels: two 16-byte loads per expert row, one 16-byte bf16 store.
 __global__ void __launch_bounds__(256) combine_kernel(
     const float* __restrict__ o, int splits, size_t split_stride, const float* __restrict__ topk_w,
     const int32_t* __restrict__ inv_row, int k_max, int64_t rcap,
@@ -109,7 +124,7 @@ __global__ void __launch_bounds__(256) combine_kernel(
   pdl_trigger();   // let the next kernel launch
   __shared__ int rows[kMaxK];
   __shared__ float wts[kMaxK];
-  const int nv = d / 4;
+  const int nv = d / 8;
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     if (threadIdx.x < k_max) {
@@ -124,34 +139,34 @@ __global__ void __launch_bounds__(256) combine_kernel(
     __syncthreads();
     const int64_t srow = shared_src ? (int64_t)(shared_row0 ? *shared_row0 : 0) + t : -1;
     for (int i = threadIdx.x; i < nv; i += blockDim.x) {
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int j = 0; j < k_max; ++j) {
         const int r = rows[j];
         if (r < 0) continue;
-        float4 v = reinterpret_cast<const float4*>(o + (size_t)r * d)[i];
-        for (int s = 1; s < splits; ++s) {
-          const float4 u = reinterpret_cast<const float4*>(o + s * split_stride + (size_t)r * d)[i];
-          v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
-        }
+        float v[8];
+        load8_rows(o, splits, split_stride, r, d, i, v);
         const float w = wts[j];
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] = fmaf(w, v[c], acc[c]);
       }
       if (srow >= 0) {
-        for (int s = 0; s < shared_splits; ++s) {
-          const float4 u = reinterpret_cast<const float4*>(
-              shared_src + s * shared_split_stride + (size_t)srow * d)[i];
-          acc.x += u.x; acc.y += u.y; acc.z += u.z; acc.w += u.w;
-        }
+        float v[8];
+        load8_rows(shared_src, shared_splits, shared_split_stride, srow, d, i, v);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[c] += v[c];
       }
-      const uint32_t lo = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.x))) |
-                          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.y))) << 16);
-      const uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.z))) |
-                          (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc.w))) << 16);
-      reinterpret_cast<uint2*>(y + (size_t)t * d)[i] = make_uint2(lo, hi);
-      if (y_f32) reinterpret_cast<float4*>(y_f32 + (size_t)t * d)[i] = acc;
+      uint32_t pk[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        pk[q] = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q]))) |
+                (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q + 1])))
+                 << 16);
+      reinterpret_cast<uint4*>(y + (size_t)t * d)[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      if (y_f32) {
+        float4* yf = reinterpret_cast<float4*>(y_f32 + (size_t)t * d) + 2 * i;
+        yf[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        yf[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      }
     }
   }
 }
@@ -211,9 +226,9 @@ cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t spl
                            const int32_t* shared_row0, int shared_splits, uint16_t* y,
                            float* y_f32, cudaStream_t s) {
   // status pointer: the combine of the split entry point has no workspace; pass none
-  launch_pdl(combine_kernel, dim3(row_grid(p.T)), dim3(256), 0, s, o, splits, split_stride, topk_w, inv_row, p.k_max,
-                                               p.Rcap, shared_src, shared_row0, shared_splits,
-                                               split_stride, p.T, p.d, y, y_f32, nullptr);
+  launch_pdl(combine_kernel, dim3(row_grid(p.T)), dim3(256), 0, s, o, splits,
+             split_stride, topk_w, inv_row, p.k_max, p.Rcap, shared_src, shared_row0,
+             shared_splits, split_stride, p.T, p.d, y, y_f32, nullptr);
   return cudaGetLastError();
 }
 
