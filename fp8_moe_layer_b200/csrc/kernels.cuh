@@ -9,7 +9,8 @@
 namespace moe {
 
 constexpr int kBK = 128;            // bytes (= e4m3 elements) of K per pipeline stage
-constexpr int kRouterTile = 32;     // router logits tile: 32 tokens x 32 experts x 32 of d
+// CUDA-core router logits tile: 64 tokens x 64 experts, d in chunks of 16
+constexpr int kRtTok = 64, kRtExp = 64, kRtK = 16;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxK = 32;
 

@@ -52,9 +52,13 @@ static int choose_splits(int64_t base_tiles, int num_kb, int units, double w_til
 }
 
 int router_splits(int T, int d, int E, int* chunks_per_split) {
-  const int64_t rtiles = ceil_div(std::max(T, 1), kRouterTile) * ceil_div(E, kRouterTile);
-  const int nchunks = (int)ceil_div(d, kRouterTile);
-  const int rs = (int)std::min<int64_t>(nchunks, std::max<int64_t>(1, ceil_div(2 * kPlanSMs, rtiles)));
+  const int64_t rtiles = ceil_div(std::max(T, 1), kRtTok) * ceil_div(E, kRtExp);
+  const int nchunks = (int)ceil_div(d, kRtK);
+  // about two waves of tiles, but at most 8192 partial logits per token for the top-k kernel
+  // to add up
+  const int64_t waves2 = std::max<int64_t>(1, ceil_div(2 * kPlanSMs, rtiles));
+  const int64_t cap = std::max<int64_t>(1, 8192 / E);
+  const int rs = (int)std::min<int64_t>(nchunks, std::min(waves2, cap));
   *chunks_per_split = (int)ceil_div(nchunks, rs);
   return (int)ceil_div(nchunks, *chunks_per_split);
 }
@@ -108,11 +112,11 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   p->slabs1 = p->pair1 ? MOE_FORCE_SLABS : 1;
 #endif
 
-  // router: 32x32 tiles; split d so that the grid covers about two waves (the tensor-core router
-  // writes whole logits)
+  // router: 64 x 64 tiles; split d so that the grid covers about two waves (the tensor-core
+  // router writes whole logits)
   if (router_uses_mma(E, T, d)) {
     p->r_splits = 1;
-    p->r_chunks_per_split = (int)ceil_div(d, kRouterTile);
+    p->r_chunks_per_split = (int)ceil_div(d, kRtK);
   } else {
     p->r_splits = router_splits(T, d, E, &p->r_chunks_per_split);
   }

@@ -97,48 +97,83 @@ __device__ __forceinline__ double dot8_f64(const uint4 v, const float4 a, const 
 }
 
 // part[s][t][e] = sum over the d-chunks of split s of x[t, d] * W[e, d], fp64, d ascending.
-// Block: 256 threads computing a 32-token x 32-expert tile; thread (ty, tx) owns tokens
-// 4*ty .. 4*ty+3 of expert tx. The tiles hold the inputs as fp64 (exact conversions).
+// Block: 256 threads computing a 64-token x 64-expert tile; thread (ty, tx) = (tid / 16,
+// tid % 16) owns tokens ty + 16 i and experts tx + 16 j (i, j < 4). d goes by chunks of 16: the
+// next chunk's inputs are loaded into registers while the current one is multiplied from shared
+// memory, where both tiles sit as fp64 (exact conversions, once per element and block), K-major
+// and double-buffered. Per chunk step a thread reads 4 token and 4 weight values for 16 fma.
 __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
                                                             const float* __restrict__ W, int T,
                                                             int d, int E, int chunks_per_split,
                                                             double* __restrict__ part) {
   pdl_wait();      // predecessor kernel complete, its writes visible
   pdl_trigger();   // let the next kernel launch
-  __shared__ double xs[kRouterTile][kRouterTile + 1];
-  __shared__ double ws[kRouterTile][kRouterTile + 1];
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const int t0 = blockIdx.x * kRouterTile, e0 = blockIdx.y * kRouterTile;
+  __shared__ __align__(16) double xs[2][kRtK][kRtTok];
+  __shared__ __align__(16) double ws[2][kRtK][kRtExp];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int t0 = blockIdx.x * kRtTok, e0 = blockIdx.y * kRtExp;
   const int split = blockIdx.z;
-  const int nchunks = (d + kRouterTile - 1) / kRouterTile;
+  const int nchunks = d / kRtK;
   const int c_begin = split * chunks_per_split;
   const int c_end = min(nchunks, c_begin + chunks_per_split);
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  for (int c = c_begin; c < c_end; ++c) {
-    const int dbase = c * kRouterTile;
+  // loader: row lr (token / expert of the tile) and 4 consecutive d of the chunk
+  const int lr = tid >> 2, lk = 4 * (tid & 3);
+  const bool tok_ok = t0 + lr < T, exp_ok = e0 + lr < E;
+  const uint16_t* xrow = x + (size_t)(tok_ok ? t0 + lr : 0) * d + lk;
+  const float* wrow = W + (size_t)(exp_ok ? e0 + lr : 0) * d + lk;
+  uint2 xv = make_uint2(0u, 0u);
+  float4 wv = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto fetch = [&](int c) {
+    if (tok_ok) xv = *reinterpret_cast<const uint2*>(xrow + (size_t)c * kRtK);
+    if (exp_ok) wv = *reinterpret_cast<const float4*>(wrow + (size_t)c * kRtK);
+  };
+  auto park = [&](int buf) {
+    xs[buf][lk + 0][lr] = static_cast<double>(__uint_as_float(xv.x << 16));
+    xs[buf][lk + 1][lr] = static_cast<double>(__uint_as_float(xv.x & 0xFFFF0000u));
+    xs[buf][lk + 2][lr] = static_cast<double>(__uint_as_float(xv.y << 16));
+    xs[buf][lk + 3][lr] = static_cast<double>(__uint_as_float(xv.y & 0xFFFF0000u));
+    ws[buf][lk + 0][lr] = static_cast<double>(wv.x);
+    ws[buf][lk + 1][lr] = static_cast<double>(wv.y);
+    ws[buf][lk + 2][lr] = static_cast<double>(wv.z);
+    ws[buf][lk + 3][lr] = static_cast<double>(wv.w);
+  };
+  double acc[4][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = ty + 8 * i;            // row of the tile this thread loads
-      const int dd = dbase + tx;
-      const int t = t0 + r, e = e0 + r;
-      xs[r][tx] = (t < T && dd < d) ? static_cast<double>(bf16_bits_to_float(x[(size_t)t * d + dd])) : 0.0;
-      ws[r][tx] = (e < E && dd < d) ? static_cast<double>(W[(size_t)e * d + dd]) : 0.0;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kRouterTile; ++kk) {
-      const double w = ws[tx][kk];
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i] = fma(xs[4 * ty + i][kk], w, acc[i]);
-    }
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  if (c_begin < c_end) {
+    fetch(c_begin);
+    park(0);
     __syncthreads();
+    for (int c = c_begin; c < c_end; ++c) {
+      const int buf = (c - c_begin) & 1;
+      if (c + 1 < c_end) fetch(c + 1);
+#pragma unroll
+      for (int kk = 0; kk < kRtK; ++kk) {
+        double xa[4], wb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xa[i] = xs[buf][kk][ty + 16 * i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) wb[j] = ws[buf][kk][tx + 16 * j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fma(xa[i], wb[j], acc[i][j]);
+      }
+      if (c + 1 < c_end) park(buf ^ 1);
+      __syncthreads();
+    }
   }
-  const int e = e0 + tx;
-  if (e < E) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = t0 + 4 * ty + i;
-      if (t < T) part[((size_t)split * T + t) * E + e] = acc[i];
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty + 16 * i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx + 16 * j;
+      if (e < E) part[((size_t)split * T + t) * E + e] = acc[i][j];
     }
   }
 }
@@ -671,8 +706,7 @@ cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float
 
 cudaError_t launch_router_logits(const Plan& p, const uint16_t* hidden, const float* router_w,
                                  double* part, cudaStream_t s) {
-  dim3 grid((p.T + kRouterTile - 1) / kRouterTile, (p.E + kRouterTile - 1) / kRouterTile,
-            p.r_splits);
+  dim3 grid((p.T + kRtTok - 1) / kRtTok, (p.E + kRtExp - 1) / kRtExp, p.r_splits);
   launch_pdl(router_logits_kernel, dim3(grid), dim3(256), 0, s, hidden, router_w, p.T, p.d, p.E,
                                             p.r_chunks_per_split, part);
   return cudaGetLastError();
