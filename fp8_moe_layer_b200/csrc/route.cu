@@ -67,6 +67,40 @@ __device__ __forceinline__ void warp_select_desc(int n, int kt, ValFn val, IdFn 
   }
 }
 
+// Block-wide descending sort of n <= kMaxExperts (value, id) pairs (equal values: lower id
+// first, the order warp_select_desc produces) into sv / si, bitonic over the next power of two
+// (padding: -inf, id INT_MAX). For selections with a large k_t, where the warp selection's k_t
+// dependent rounds are the kernel's critical path. Every thread of the block calls it.
+template <typename ValFn, typename IdFn>
+__device__ void block_sort_desc(int n, ValFn val, IdFn idf, double* sv, int* si) {
+  int np = 1;
+  while (np < n) np <<= 1;
+  for (int i = threadIdx.x; i < np; i += blockDim.x) {
+    sv[i] = i < n ? val(i) : -INFINITY;
+    si[i] = i < n ? idf(i) : 0x7FFFFFFF;
+  }
+  __syncthreads();
+  for (int k = 2; k <= np; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < np; i += blockDim.x) {
+        const int q = i ^ j;
+        if (q > i) {
+          const double a = sv[i], b = sv[q];
+          const int ia = si[i], ib = si[q];
+          const bool a_first = a > b || (a == b && ia < ib);
+          if (a_first != ((i & k) == 0)) {
+            sv[i] = b;
+            sv[q] = a;
+            si[i] = ib;
+            si[q] = ia;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 // Renormalised weights of the selection held by lanes j < kt (sel_v descending): fp64
 // exp(l_j - l_max) / sum, rounded once to fp32; ids and weights of slots >= kt are -1 and 0.
 __device__ __forceinline__ void warp_store_selection(double sel_v, int sel_e, int kt, int k_max,
@@ -93,6 +127,28 @@ __device__ __forceinline__ double dot8_f64(const uint4 v, const float4 a, const 
   c = fma(static_cast<double>(__uint_as_float(v.z & 0xFFFF0000u)), static_cast<double>(b.y), c);
   c = fma(static_cast<double>(__uint_as_float(v.w << 16)), static_cast<double>(b.z), c);
   c = fma(static_cast<double>(__uint_as_float(v.w & 0xFFFF0000u)), static_cast<double>(b.w), c);
+  return c;
+}
+
+// Eight bf16 values (one 16-byte load) as fp64 (exact), in order.
+__device__ __forceinline__ void bf16x8_to_f64(const uint4 v, double (&o)[8]) {
+  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    o[2 * q] = static_cast<double>(__uint_as_float(w4[q] << 16));
+    o[2 * q + 1] = static_cast<double>(__uint_as_float(w4[q] & 0xFFFF0000u));
+  }
+}
+// sum_j x[j] * w[j] for eight fp64 token values and eight fp32 weights, in the order of dot8_f64.
+__device__ __forceinline__ double dot8_xw(const double (&x)[8], const float4 a, const float4 b) {
+  double c = x[0] * static_cast<double>(a.x);
+  c = fma(x[1], static_cast<double>(a.y), c);
+  c = fma(x[2], static_cast<double>(a.z), c);
+  c = fma(x[3], static_cast<double>(a.w), c);
+  c = fma(x[4], static_cast<double>(b.x), c);
+  c = fma(x[5], static_cast<double>(b.y), c);
+  c = fma(x[6], static_cast<double>(b.z), c);
+  c = fma(x[7], static_cast<double>(b.w), c);
   return c;
 }
 
@@ -188,8 +244,8 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __re
 //  refine (refine_w != null, for the tensor-core logits): the approximate logits only pick the
 //         candidates -- every expert within kRefineWindow of the approximate k_t-th largest, which
 //         contains the exact top-k_t while the approximation error stays below half the window --
-//         and each candidate's logit is recomputed in fp64 (one warp per candidate) before the
-//         selection and the weights.
+//         and each candidate's logit is recomputed in fp64 before the selection and the weights
+//         (a warp takes two candidates, so each token value is converted once for both).
 constexpr double kRefineWindow = 1e-2;
 constexpr int kMaxCandidates = 256;
 
@@ -204,6 +260,8 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
   __shared__ double lg[kMaxExperts];
   __shared__ float red[4];
   __shared__ int cand[kMaxCandidates];
+  __shared__ double sort_v[kMaxExperts];
+  __shared__ int sort_i[kMaxExperts];
   __shared__ int ncand;
   __shared__ double vk_s;
   const int t = blockIdx.x;
@@ -232,8 +290,16 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
       kt = max(1, min(kt, kcap));
     }
     bool by_cand = false;          // exact selection over the refined candidates only
+    // large k_t: a block-wide sort instead of k_t rounds of the warp selection
+    const bool sort_all = kt > 8 && E > 64;
     if (refine_w) {
-      if (warp == 0) {
+      if (sort_all) {
+        block_sort_desc(E, [&](int c) { return lg[c]; }, [](int c) { return c; }, sort_v, sort_i);
+        if (tid == 0) {
+          vk_s = sort_v[kt - 1];                                   // approximate k_t-th largest
+          ncand = 0;
+        }
+      } else if (warp == 0) {
         double sv;
         int se;
         warp_select_desc(E, kt, [&](int c) { return lg[c]; }, [](int c) { return c; }, sv, se);
@@ -256,20 +322,46 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
       const int nc = all ? E : ncand;
       const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
       const int nv = d / 8;
-      for (int c = warp; c < nc; c += 4) {
-        const int e = all ? c : cand[c];
-        const float4* wr = reinterpret_cast<const float4*>(refine_w + (size_t)e * d);
-        double acc = 0.0;
-#pragma unroll 4
-        for (int i = lane; i < nv; i += 32) acc += dot8_f64(xr[i], __ldg(wr + 2 * i), __ldg(wr + 2 * i + 1));
+      for (int c0 = 2 * warp; c0 < nc; c0 += 8) {
+        const bool two = c0 + 1 < nc;
+        const int e0 = all ? c0 : cand[c0];
+        const int e1 = two ? (all ? c0 + 1 : cand[c0 + 1]) : e0;
+        const float4* w0 = reinterpret_cast<const float4*>(refine_w + (size_t)e0 * d);
+        const float4* w1 = reinterpret_cast<const float4*>(refine_w + (size_t)e1 * d);
+        double acc0 = 0.0, acc1 = 0.0;
+#pragma unroll 2
+        for (int i = lane; i < nv; i += 32) {
+          double xv[8];
+          bf16x8_to_f64(xr[i], xv);
+          acc0 += dot8_xw(xv, __ldg(w0 + 2 * i), __ldg(w0 + 2 * i + 1));
+          if (two) acc1 += dot8_xw(xv, __ldg(w1 + 2 * i), __ldg(w1 + 2 * i + 1));
+        }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) lg[e] = acc + (bias ? static_cast<double>(bias[e]) : 0.0);
+        for (int off = 16; off > 0; off >>= 1) {
+          acc0 += __shfl_xor_sync(0xffffffffu, acc0, off);
+          acc1 += __shfl_xor_sync(0xffffffffu, acc1, off);
+        }
+        if (lane == 0) {
+          lg[e0] = acc0 + (bias ? static_cast<double>(bias[e0]) : 0.0);
+          if (two) lg[e1] = acc1 + (bias ? static_cast<double>(bias[e1]) : 0.0);
+        }
       }
       __syncthreads();
       by_cand = !all;
     }
-    if (warp == 0) {
+    const int nsel = by_cand ? ncand : E;
+    if (kt > 8 && nsel > 64) {
+      if (by_cand)
+        block_sort_desc(ncand, [&](int c) { return lg[cand[c]]; }, [&](int c) { return cand[c]; },
+                        sort_v, sort_i);
+      else
+        block_sort_desc(E, [&](int c) { return lg[c]; }, [](int c) { return c; }, sort_v, sort_i);
+      if (warp == 0) {
+        const double sv = lane < kt ? sort_v[lane] : 0.0;
+        const int se = lane < kt ? sort_i[lane] : -1;
+        warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
+      }
+    } else if (warp == 0) {
       double sv;
       int se;
       if (by_cand)
