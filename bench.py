@@ -40,10 +40,11 @@ sys.path.insert(0, ROOT)
 WORKLOAD = "deepseek_T8192"
 METRIC = "MoE-layer µs and tokens/s at 1 B200; % of HBM (decode) / FP8 TC (prefill) roofline"
 FLUSH_BYTES = 256 << 20
-# A ~0.2 ms GPU sleep (cycles at ~2 GHz) before each timed step: the host enqueues the step's
-# kernels (tens of microseconds of launches) while the GPU sleeps, so the events measure device
-# time and not the host's launch rate. The host cost is in the e2e number.
-HOST_AHEAD_CYCLES = 400_000
+# A ~1 ms GPU sleep (cycles at ~2 GHz) before each timed step: the host enqueues the step's
+# kernels (tens to hundreds of microseconds of launches and argument set-up) while the GPU
+# sleeps, so the events measure device time and not the host's launch rate. The host cost is in
+# the e2e number.
+HOST_AHEAD_CYCLES = 2_000_000
 # nominal B200 figures: HBM3e bandwidth, dense FP8 tensor-core throughput; FP8 / bf16 ratio
 NOMINAL_HBM_GBS = 8000.0
 NOMINAL_FP8_TFLOPS = 4500.0

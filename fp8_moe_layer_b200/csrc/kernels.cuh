@@ -92,7 +92,7 @@ cudaError_t launch_topk_quant(const Plan& p, const double* part, const float* bi
 // logits + topk_quant.
 // (the fused router holds a token's row in registers: d <= 8192)
 inline bool router_is_fused(int E, int d) { return E <= 32 && d <= 8192; }
-// Router logits on the tensor cores (three bf16 planes + exact refinement of the candidates) once
+// Router logits on the tensor cores (two bf16 planes + exact refinement of the candidates) once
 // the fp32 CUDA-core work 2·T·E·d is large: measured on B200, the exact CUDA-core router is faster
 // up to T·E·d ~ 2.4e8 (Qwen3 T=64, DeepSeek T=128, MoE-Prism T=64) and the tensor-core one from
 // ~1.1e9 (Qwen3 T=4096, MoE-Prism T=2048, DeepSeek T=8192); the switch sits at 2^29.
@@ -125,7 +125,7 @@ cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float
                               cudaStream_t s);
 // Tokens per tile of the tensor-core router (64 or 128): the box height of map_x.
 int router_mma_tokens(int T, int E);
-// planes: 3 * E * d bf16 (workspace); map_w over planes [3][E][d], map_x over hidden [T][d]
+// planes: 2 * E * d bf16 (workspace); map_w over planes [2][E][d], map_x over hidden [T][d]
 cudaError_t launch_router_mma(const Plan& p, const float* router_w, uint16_t* planes,
                               const CUtensorMap& map_w, const CUtensorMap& map_x, double* logits,
                               int* status, cudaStream_t s);

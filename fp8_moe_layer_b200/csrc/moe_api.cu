@@ -165,7 +165,7 @@ int plan_make(int T, int d, int E, int F, int k_max, int Fs, Plan* p, int k_est)
   p->off_aq = take((size_t)p->Rpad * F);
   p->off_s2 = take(sizeof(float) * (size_t)p->Rpad);
   p->off_o = take(sizeof(float) * (size_t)p->g2_splits * p->Rpad * d);
-  p->off_planes = take(router_uses_mma(E, T, d) ? 3 * sizeof(uint16_t) * (size_t)E * d : 0);
+  p->off_planes = take(router_uses_mma(E, T, d) ? 2 * sizeof(uint16_t) * (size_t)E * d : 0);
   p->off_hpart = take(p->g1_splits > 1 ? sizeof(float) * p->g1_splits * (size_t)p->Rcap * 2 * F : 0);
   p->bytes = off;
   return MOE_OK;
@@ -221,9 +221,9 @@ static bool map_out(CUtensorMap* m, const float* o, int64_t rows, int d) {
                   CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// bf16 router weight planes [3][E][d]: box 64 (K) x 128 experts of one plane.
+// bf16 router weight planes [2][E][d]: box 64 (K) x 128 experts of one plane.
 static bool map_router_planes(CUtensorMap* m, const uint16_t* planes, int E, int d) {
-  const uint64_t dims[3] = {(uint64_t)d, (uint64_t)E, 3};
+  const uint64_t dims[3] = {(uint64_t)d, (uint64_t)E, 2};
   const uint64_t str[2] = {(uint64_t)d * 2, (uint64_t)E * d * 2};
   const uint32_t box[3] = {64, 128, 1};
   return make_map(m, planes, 3, dims, str, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);

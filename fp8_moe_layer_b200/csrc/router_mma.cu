@@ -1,17 +1,18 @@
 // Router logits on the tensor cores for large E and T: l[t, e] = sum_d x[t, d] W[e, d].
 //
-// x is bf16 (exact); the fp32 router weights are split exactly into three bf16 planes,
-// W = hi + mid + lo (hi = bf16(W), mid = bf16(W - hi), lo = W - hi - mid; 3 x 8 significand
-// bits cover fp32's 24, and each difference is exact in fp32). Every product x * plane is exact
-// in fp32, so three tcgen05.mma kind::f16 (bf16 x bf16 -> fp32) per K-step give logits with the
-// accuracy of an fp32 dot product at tensor-core speed.
+// x is bf16 (exact); the fp32 router weights are split into two bf16 planes, W ~ hi + mid
+// (hi = bf16(W), mid = bf16(W - hi): 16 of fp32's 24 significand bits, |W - hi - mid| <=
+// 2^-18 |W|). Every product x * plane is exact in fp32, so two tcgen05.mma kind::f16
+// (bf16 x bf16 -> fp32) per K-step give logits within 2^-18 sum|x W| plus the fp32 accumulation
+// error of the exact ones. They only pick the candidates that the top-k kernel recomputes in
+// fp64: an error far below half of its candidate window is all they need.
 //
 // Method: "Routage MoE entre GPU" (viite.ai): the router scores every expert from the token's
 // hidden state. The top-k and the weights follow in topk_quant_kernel (route.cu).
 //
 // Tiles: 128 experts (MMA M, TMEM lanes) x NT tokens (MMA N, 64 or 128); K-step = 64 bf16 = one
-// 128-byte swizzled row. One stage holds the three weight planes and the token tile (56 or 64 KB;
-// four or three stages). 128-token tiles halve the weight bytes per MMA; they are used when they
+// 128-byte swizzled row. One stage holds the two weight planes and the token tile (40 or 48 KB;
+// five or four stages). 128-token tiles halve the weight bytes per MMA; they are used when they
 // still give about a wave of tiles (DeepSeek-V3 T=8192: 128 tiles instead of 1.7 waves of 64).
 // Persistent grid, one CTA per SM, warp 0 = TMA producer, warp 1 = MMA issuer, warp 2 = TMEM
 // allocator, warps 4-7 = epilogue (fp32 logits, coalesced over experts). Bounded waits as in
@@ -22,11 +23,12 @@
 namespace moe {
 
 constexpr int kRtPlaneBytes = 128 * kBK;         // 128 experts x 64 bf16
+constexpr int kRtPlanes = 2;                      // bf16 planes of the router weights
 template <int NT>
 struct RtCfg {
   static constexpr int B_BYTES = NT * kBK;                       // NT tokens x 64 bf16
-  static constexpr int STAGE_BYTES = 3 * kRtPlaneBytes + B_BYTES;
-  static constexpr int STAGES = NT == 64 ? 4 : 3;
+  static constexpr int STAGE_BYTES = kRtPlanes * kRtPlaneBytes + B_BYTES;
+  static constexpr int STAGES = NT == 64 ? 5 : 4;
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
 };
 
@@ -45,7 +47,7 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
-// planes[p][e][d], p = 0 hi, 1 mid, 2 lo.
+// planes[p][e][d], p = 0 hi, 1 mid.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ W, int64_t n,
                                                            uint16_t* __restrict__ planes) {
   pdl_wait();      // predecessor kernel complete, its writes visible
@@ -55,11 +57,8 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
     const __nv_bfloat16 hi = __float2bfloat16_rn(w);
     const float r1 = w - __bfloat162float(hi);
     const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
     planes[i] = __bfloat16_as_ushort(hi);
     planes[n + i] = __bfloat16_as_ushort(mid);
-    planes[2 * n + i] = __bfloat16_as_ushort(lo);
   }
 }
 
@@ -123,9 +122,9 @@ __global__ void __launch_bounds__(256, 1)
           }
           uint8_t* st = smem + stage * kRtStageBytes;
           mbar_arrive_expect_tx(&full[stage], kRtStageBytes);
-          for (int p = 0; p < 3; ++p)
+          for (int p = 0; p < kRtPlanes; ++p)
             tma_load_3d(st + p * kRtPlaneBytes, &map_w, &full[stage], kb * 64, m * 128, p, pol);
-          tma_load_2d(st + 3 * kRtPlaneBytes, &map_x, &full[stage], kb * 64, n * kRtN, pol);
+          tma_load_2d(st + kRtPlanes * kRtPlaneBytes, &map_x, &full[stage], kb * 64, n * kRtN, pol);
           ++issued;
           if (++stage == kRtStages) {
             stage = 0;
@@ -166,9 +165,9 @@ __global__ void __launch_bounds__(256, 1)
           }
           tc_fence_after_sync();
           const uint32_t st = smem_addr(smem + stage * kRtStageBytes);
-          const uint64_t bdesc = smem_desc_sw128(st + 3 * kRtPlaneBytes);
+          const uint64_t bdesc = smem_desc_sw128(st + kRtPlanes * kRtPlaneBytes);
 #pragma unroll
-          for (int p = 0; p < 3; ++p) {
+          for (int p = 0; p < kRtPlanes; ++p) {
             const uint64_t adesc = smem_desc_sw128(st + p * kRtPlaneBytes);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)          // K = 16 bf16 (32 bytes) per instruction
