@@ -117,6 +117,8 @@ struct DecodeGrouping {
   int32_t* tiles;
   uint32_t* amax;
   int BN, has_shared;
+  uint8_t* xqp;     // gathered FP8 rows [rows][d] (with the quantisation), or null
+  float* xsp;       // their scales [rows]
 };
 cudaError_t launch_route_gemv(const Plan& p, const uint16_t* hidden, const float* router_w,
                               const float* bias, int k, const int32_t* k_per_token,

@@ -651,7 +651,8 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
   } else if (router_uses_gemv(p)) {
     // decode batch: logits, top-k, quantisation and the grouping in one kernel (the events of
     // stages 1 and 2 bracket nothing)
-    const DecodeGrouping grp{w.offsets, w.perm, w.inv, w.tiles, w.amax, p.BN, p.shared ? 1 : 0};
+    const DecodeGrouping grp{w.offsets, w.perm, w.inv, w.tiles, w.amax, p.BN, p.shared ? 1 : 0,
+                             w.xqp, w.xsp};
     MOE_CUDA(launch_route_gemv(p, hidden, router_w, router_bias, k, k_per_token, w.part, w.ids,
                                w.w, w.xq, w.xs, true, w.status, grp, s));
     record(1);
@@ -663,10 +664,11 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
                                w.status, s));
   }
   record(2);
-  // grouping: by the decode router itself (T <= 8), with the row gather in one kernel
-  // (T * k_max <= 8192), or alone; the gather kernel follows in the last two cases
+  // grouping and row gather: by the decode router itself (T <= 8), in one kernel
+  // (T * k_max <= 8192), or the grouping kernels followed by the gather kernel
   bool gathered = false;
   if (router_uses_gemv(p)) {
+    gathered = true;                 // the decode router also gathered the rows
   } else if (!permute_gather_fused(p)) {
     MOE_CUDA(launch_permute(p, w.ids, k, k_per_token, w.offsets, w.perm, w.inv, w.tiles, w.pscr,
                             w.status, s));

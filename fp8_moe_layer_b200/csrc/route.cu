@@ -622,6 +622,20 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
         out[i] = make_uint2(packed[0], packed[1]);
       }
     }
+    if (grp.offsets && grp.xqp) {
+      // the row gather of the grouped FFN: xqp[r, :] = xq[perm[r], :], xsp[r] = xs[perm[r]] for
+      // the routed rows and the shared expert's (this block wrote perm, xq and xs)
+      __syncthreads();
+      const int rows = grp.offsets[E] + (grp.has_shared ? T : 0);
+      const int n16 = d / 16;
+      for (int i = tid; i < rows * n16; i += 256) {
+        const int r = i / n16, c = i - r * n16;
+        const int t = grp.perm[r];
+        reinterpret_cast<uint4*>(grp.xqp + (size_t)r * d)[c] =
+            reinterpret_cast<const uint4*>(xq + (size_t)t * d)[c];
+      }
+      for (int r = tid; r < rows; r += 256) grp.xsp[r] = xs[grp.perm[r]];
+    }
   }
   if (tid == 0) status[3] = 0;             // the counter is ready for the next launch
 }
