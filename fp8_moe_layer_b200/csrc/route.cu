@@ -492,6 +492,11 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // the selection, kept in shared memory for the grouping and the gather (-1: unused slot)
+  __shared__ int s_ids[kGemvMaxT * kMaxK];
+  __shared__ int s_inv[kGemvMaxT * kMaxK];
+  __shared__ int s_kt[kGemvMaxT];
+  __shared__ int s_R;
   if (warp < T) {
     const int t = warp;
     double* my = lgd + (size_t)t * E;
@@ -507,13 +512,15 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
     int se;
     warp_select_desc(E, kt, [&](int c) { return my[c]; }, [](int c) { return c; }, sv, se);
     warp_store_selection(sv, se, kt, k_max, ids + (size_t)t * k_max, wout + (size_t)t * k_max);
+    if (lane < k_max) s_ids[t * k_max + lane] = lane < kt ? se : -1;
+    if (lane == 0) s_kt[t] = kt;
   }
+  __syncthreads();                                     // the selection of every token
   if (grp.offsets) {
     // The grouping of the (at most 8 x 32) routed pairs, by this block: expert counts, their
     // exclusive prefix (offsets), each pair's row = offset + its rank among the earlier pairs of
     // the same expert (token-major order: stable), and the GEMM tile prefix. Same result as the
     // grouping kernels (permute.cu); it also zeroes the rows' SwiGLU maxima.
-    __syncthreads();                                   // ids of every token written
     __shared__ int tmp[9];
     int* cnt = reinterpret_cast<int*>(lgd);            // [E] (the logit copies are done with)
     int* off = cnt + E;                                // [E]
@@ -522,10 +529,7 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
     const int npairs = T * k_max;                      // <= 8 * 32 = 256 = blockDim
     int my_e = -1;
     if (tid < npairs) {
-      const int t = tid / k_max, j = tid % k_max;
-      int kt = k_per_token ? k_per_token[t] : k;
-      kt = max(1, min(kt, min(E, k_max)));
-      const int e = j < kt ? ids[tid] : -1;
+      const int e = s_ids[tid];
       if (e >= 0 && e < E) {
         my_e = e;
         atomicAdd(&cnt[e], 1);
@@ -554,19 +558,16 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
       int row = -1;
       if (my_e >= 0) {
         int rank = 0;
-        for (int i = 0; i < tid; ++i) {
-          const int ti = i / k_max, ji = i % k_max;
-          int kti = k_per_token ? k_per_token[ti] : k;
-          kti = max(1, min(kti, min(E, k_max)));
-          if (ji < kti && ids[i] == my_e) ++rank;
-        }
+        for (int i = 0; i < tid; ++i) rank += s_ids[i] == my_e ? 1 : 0;
         row = off[my_e] + rank;
         grp.perm[row] = tid / k_max;
         grp.amax[row] = 0u;
       }
       grp.inv[tid] = row;
+      s_inv[tid] = row;
     }
     if (tid == 0) {
+      s_R = R;
       grp.offsets[E] = R;
       grp.tiles[E] = total_tiles;
       if (grp.has_shared) {
@@ -578,34 +579,57 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
       grp.perm[R + tid] = tid;
       grp.amax[R + tid] = 0u;
     }
+    __syncthreads();                                   // s_inv, s_R
   }
   if (do_quant) {
-    // the FP8 quantisation of each token by the whole block
-    __shared__ float red[8];
-    for (int t = 0; t < T; ++t) {
-      const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-      float amax = 0.f;
-      for (int i = tid; i < nv; i += 256) {
-        const uint4 v = xr[i];
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    // The FP8 quantisation of each token by the whole block: the row maxima of all tokens in one
+    // pass (every token's loads in flight), then the codes, written to the token's row of xq
+    // and, with the grouping, straight to its routed rows (and shared-expert row) of the
+    // gathered copy, with their scales.
+    __shared__ float s_am[8][kGemvMaxT];
+    float am[TT];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] << 16)));
-          amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] & 0xFFFF0000u)));
+    for (int t = 0; t < TT; ++t) am[t] = 0.f;
+    for (int i = tid; i < nv; i += 256) {
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        if (t < T) {
+          const uint4 v = reinterpret_cast<const uint4*>(x + (size_t)t * d)[i];
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            am[t] = fmaxf(am[t], fabsf(__uint_as_float(w4[q] << 16)));
+            am[t] = fmaxf(am[t], fabsf(__uint_as_float(w4[q] & 0xFFFF0000u)));
+          }
         }
       }
+    }
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-      if (lane == 0) red[warp] = amax;
-      __syncthreads();
-      float am = red[0];
+        am[t] = fmaxf(am[t], __shfl_xor_sync(0xffffffffu, am[t], off));
+      if (lane == 0 && t < T) s_am[warp][t] = am[t];
+    }
+    __syncthreads();
+    const bool gather = grp.offsets && grp.xqp;
+    for (int t = 0; t < T; ++t) {
+      float amx = s_am[0][t];
 #pragma unroll
-      for (int w = 1; w < 8; ++w) am = fmaxf(am, red[w]);
-      __syncthreads();                                   // red[] is reused by the next token
-      const float sc = am > 0.f ? __fdiv_rn(am, 448.f) : 1.f;
-      if (tid == 0) xs[t] = sc;
-      uint2* out = reinterpret_cast<uint2*>(xq + (size_t)t * d);
+      for (int w = 1; w < 8; ++w) amx = fmaxf(amx, s_am[w][t]);
+      const float sc = amx > 0.f ? __fdiv_rn(amx, 448.f) : 1.f;
+      const int kt = s_kt[t];
+      if (tid == 0) {
+        xs[t] = sc;
+        if (gather) {
+          for (int j = 0; j < kt; ++j) {
+            const int r = s_inv[t * k_max + j];
+            if (r >= 0) grp.xsp[r] = sc;
+          }
+          if (grp.has_shared) grp.xsp[s_R + t] = sc;
+        }
+      }
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
       for (int i = tid; i < nv; i += 256) {
         const uint4 v = xr[i];
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -619,22 +643,16 @@ __global__ void __launch_bounds__(256) route_gemv_kernel(
           packed[q / 2] = static_cast<uint32_t>(e4m3x2(a0, a1)) |
                           (static_cast<uint32_t>(e4m3x2(a2, a3)) << 16);
         }
-        out[i] = make_uint2(packed[0], packed[1]);
+        const uint2 pk = make_uint2(packed[0], packed[1]);
+        reinterpret_cast<uint2*>(xq + (size_t)t * d)[i] = pk;
+        if (gather) {
+          for (int j = 0; j < kt; ++j) {
+            const int r = s_inv[t * k_max + j];
+            if (r >= 0) reinterpret_cast<uint2*>(grp.xqp + (size_t)r * d)[i] = pk;
+          }
+          if (grp.has_shared) reinterpret_cast<uint2*>(grp.xqp + (size_t)(s_R + t) * d)[i] = pk;
+        }
       }
-    }
-    if (grp.offsets && grp.xqp) {
-      // the row gather of the grouped FFN: xqp[r, :] = xq[perm[r], :], xsp[r] = xs[perm[r]] for
-      // the routed rows and the shared expert's (this block wrote perm, xq and xs)
-      __syncthreads();
-      const int rows = grp.offsets[E] + (grp.has_shared ? T : 0);
-      const int n16 = d / 16;
-      for (int i = tid; i < rows * n16; i += 256) {
-        const int r = i / n16, c = i - r * n16;
-        const int t = grp.perm[r];
-        reinterpret_cast<uint4*>(grp.xqp + (size_t)r * d)[c] =
-            reinterpret_cast<const uint4*>(xq + (size_t)t * d)[c];
-      }
-      for (int r = tid; r < rows; r += 256) grp.xsp[r] = xs[grp.perm[r]];
     }
   }
   if (tid == 0) status[3] = 0;             // the counter is ready for the next launch
