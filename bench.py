@@ -16,7 +16,10 @@ tokens per GPU, 11.6 GB of FP8 expert weights).
   FP8 tensor-core peak (tensor-bound workloads) or the HBM copy bandwidth (bytes-bound ones).
 * layer_roofline: t_roof = max(B_alg / BW, F_alg / P_fp8) over the measured step time, against
   the measured and the nominal (8 TB/s, 4.5 PFLOP/s) denominators.
-* other_configs: every other workload of the layer timed the same way (shorter).
+* l2_cold_check: the same layer timed with 2 to 8 copies of its weights used in turn and no L2
+  flush (median), beside the flushed median: a cross-check that the flush gives cold-L2 times.
+* other_configs: every other workload of the layer timed the same way (shorter), each with the
+  same rotated-copies cross-check.
 * cpu_baseline (rank 0, N=1): the CPU oracle's whole-layer time, estimated from a bounded sample.
 * --impl reference: the CPU oracle as the reference arm (no GPU work).
 Multi-GPU: independent replicas (one batch per rank, seed = rank), no collective on the path.
@@ -345,6 +348,42 @@ def _timed_steps(layer, hidden, kpt, y, steps, flush, flush_rd, stream, stage_ev
     return np.array([starts[i].elapsed_time(ends[i]) for i in range(steps)])
 
 
+L2_BYTES = 126 << 20
+
+
+def rotated_us(layer, hidden, kpt, y, touched_bytes, steps, stream):
+    """Cross-check of the L2-flush timing: µs / layer (median) with R copies of the layer's weights
+    used in turn and no flush, R chosen so that the weights the other copies touch between two
+    uses of one copy exceed twice the L2 (at most 8 copies). Returns (us, R)."""
+    import torch
+    from fp8_moe_layer_b200 import ops
+    R = int(min(8, max(2, np.ceil(2 * L2_BYTES / max(touched_bytes, 1)) + 1)))
+    cp = lambda t: None if t is None else t.clone()
+    reps = [(layer.router_w, layer.w13, layer.w13_scale, layer.w2, layer.w2_scale, layer.shared)]
+    for _ in range(R - 1):
+        reps.append((cp(layer.router_w), cp(layer.w13), cp(layer.w13_scale), cp(layer.w2),
+                     cp(layer.w2_scale),
+                     None if layer.shared is None else tuple(cp(t) for t in layer.shared)))
+    s = layer.shape
+    run = lambda r: ops.moe_forward(hidden, r[0], layer.router_bias, s.k, kpt, r[1], r[2], r[3],
+                                    r[4], s.k_max, shared=r[5], ws=layer.ws, y=y)
+    for i in range(2 * R):
+        run(reps[i % R])
+    n = max(steps, 2 * R)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for i in range(n):
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
+        starts[i].record(stream)
+        run(reps[i % R])
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    us = float(np.median([starts[i].elapsed_time(ends[i]) for i in range(n)])) * 1e3
+    del reps
+    torch.cuda.empty_cache()
+    return us, R
+
+
 def other_configs(main_name, main_layer, args, flush, flush_rd, stream, pk):
     """Every other workload of the layer: µs / layer (median of the steps) and its roofline
     fractions. Workloads of one layer shape share its weights (they differ in T only)."""
@@ -378,11 +417,13 @@ def other_configs(main_name, main_layer, args, flush, flush_rd, stream, pk):
             ms = _timed_steps(layer, h, kpt, y, 10, flush, flush_rd, stream)
             us = float(np.median(ms)) * 1e3
             lr = layer_roofline(work, us, pk)
+            us_rot, reps = rotated_us(layer, h, kpt, y, work["bytes"], 10, stream)
             out.append(dict(workload=s.name, T=s.T, us_per_layer=round(us, 2),
                             tokens_per_s=round(s.T / (us * 1e-6)),
                             active_experts=work["active_experts"],
                             frac_measured=lr["measured"]["frac"],
-                            binds=lr["measured"]["binds"], frac_nominal=lr["nominal"]["frac"]))
+                            binds=lr["measured"]["binds"], frac_nominal=lr["nominal"]["frac"],
+                            us_weights_rotated=round(us_rot, 2), weight_copies=reps))
             if ops.device_status(layer.ws) != ops.MOE_OK:
                 raise RuntimeError(f"device status not ok on {s.name}")
         if layer is not main_layer:
@@ -502,6 +543,12 @@ def run_ours(args):
                 tensor_frac_nominal=round(g1_tflops / NOMINAL_FP8_TFLOPS, 4))
     stages = {name: round(float(stage_ms[:, j].mean()) * 1e3, 2)
               for j, name in enumerate(ops.STAGE_NAMES)}
+    # the L2-flush timing cross-checked by rotating copies of the weights instead (one GPU)
+    l2_check = None
+    if world == 1:
+        us_rot, copies = rotated_us(layer, hidden, kpt, y, work["bytes"], args.steps, stream)
+        l2_check = dict(weight_copies=copies, us_per_layer_median=round(us_rot, 2),
+                        us_per_layer_median_flushed=round(float(np.median(step_ms)) * 1e3, 2))
     others = None
     if world == 1 and not args.no_other_configs:
         others = other_configs(args.workload, layer, args, flush, flush_rd, stream, pk)
@@ -526,6 +573,7 @@ def run_ours(args):
                             routed_rows=work["routed_rows"]),
         fp8_cublas_tflops_same_run=None if fp8_cublas is None else round(fp8_cublas, 1),
         stage_us=stages,
+        l2_cold_check=l2_check,
         e2e=dict(value=replicas.aggregate_tokens_per_s(shape.T, world, e2e_ms), unit="tokens/s",
                  h2d_bytes_per_step=shape.T * shape.d * 2, d2h_bytes_per_step=shape.T * shape.d * 2),
         gpu_launches=int(launches),
