@@ -2,9 +2,10 @@
 // dynamic FP8 e4m3 quantisation (scale = amax / 448). Four kernels, by shape:
 //   route_block_kernel   E <= 32: one block per token does all of it;
 //   route_gemv_kernel    decode batches (T <= 8, E > 32): a warp per expert, and the last block
-//                        to finish selects and quantises;
-//   router_logits_kernel fp32 CUDA-core logits (deterministic split over the hidden dimension),
-//   + topk_quant_kernel  then per token a warp-level top-k and the quantisation;
+//                        to finish selects, quantises, and (in moe_forward) groups and gathers;
+//   router_logits_kernel fp64 CUDA-core logits (64 x 64 register-blocked tiles, deterministic
+//   + topk_quant_kernel  split over the hidden dimension), then per token the top-k (a warp
+//                        selection, or a block sort for k_t > 8) and the quantisation;
 //   topk_quant_kernel    also after the tensor-core logits (router_mma.cu), refining the
 //                        candidates' logits exactly before the selection.
 //
@@ -415,10 +416,11 @@ __global__ void __launch_bounds__(128) topk_quant_kernel(
 // Decode router (T <= 8 tokens, E > 32): one warp per expert computes that expert's fp64 logit
 // for every token (lane-strided chunks of 8 along d, then a butterfly; all loads in flight),
 // writes it to `logits` [T][E], and the last block to finish (a counter in the status word,
-// status[3]) selects the top-k, the weights and the FP8 quantisation of every token, then resets
-// the counter. One kernel instead of the tiled logits kernel (one global round trip per 32-wide
-// chunk of d) plus a separate top-k kernel. Dynamic shared memory: T * E doubles (the last
-// block's copy of the logits).
+// status[3]) selects the top-k and the weights of every token, groups the routed pairs by expert
+// (when given a DecodeGrouping), quantises every token to FP8 -- writing the codes to the token
+// rows and straight to the token's routed rows of the gathered copy -- then resets the counter.
+// One kernel instead of the logits, top-k, grouping and gather kernels. Dynamic shared memory:
+// T * E doubles (the last block's copy of the logits, reused by the grouping).
 constexpr int kGemvMaxT = 8;
 
 // Exclusive prefix sum over the 256 threads of a block (tmp: 9 ints of shared memory); returns
