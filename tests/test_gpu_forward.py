@@ -72,13 +72,13 @@ SMALL = [
     # decode batches with E > 32 (the one-kernel GEMV router)
     I.MoEShape("decode_gemv_T3", 3, 256, 96, 128, 6, 6, zipf_s=1.0),
     I.MoEShape("decode_gemv_T8_shared", 8, 256, 40, 128, 4, 4, F_shared=128),
-    # at most four tokens: the grouped FFN on the CUDA cores (one to four rows per group, the
-    # shared expert's group, per-token k, K-split down pieces, E <= 32 with the fused router)
-    I.MoEShape("ffn_cuda_core_T1", 1, 256, 64, 128, 8, 8),
-    I.MoEShape("ffn_cuda_core_T2_shared", 2, 256, 40, 128, 4, 4, F_shared=128),
-    I.MoEShape("ffn_cuda_core_T4_elastic", 4, 128, 48, 64, 2, 8, k_choices=(1, 2, 4, 8)),
-    I.MoEShape("ffn_cuda_core_T3_small_E", 3, 512, 8, 1024, 2, 2),
-    I.MoEShape("ffn_cuda_core_T4_long_F", 4, 128, 4, 4096, 2, 2, F_shared=4096),
+    # one to four tokens: groups of one to four rows in 16-column token tiles, the shared
+    # expert's group, per-token k, K-split gate/up partials, E <= 32 with the fused router
+    I.MoEShape("decode_T1", 1, 256, 64, 128, 8, 8),
+    I.MoEShape("decode_T2_shared", 2, 256, 40, 128, 4, 4, F_shared=128),
+    I.MoEShape("decode_T4_elastic", 4, 128, 48, 64, 2, 8, k_choices=(1, 2, 4, 8)),
+    I.MoEShape("decode_T3_small_E", 3, 512, 8, 1024, 2, 2),
+    I.MoEShape("decode_T4_long_F", 4, 128, 4, 4096, 2, 2, F_shared=4096),
     # token tiles >= 192 rows run the gate/up GEMM on 2-SM pairs, and the down GEMM too when
     # F >= 2048: odd weight m-tile counts (F = 192 -> 3 gate/up tiles, d = 384 -> 3 down tiles;
     # the pair's second half falls off the matrix), ragged tails, a shared-expert group
