@@ -22,7 +22,7 @@ LIB_WAITTEST = os.path.join(HERE, "libfp8moe_waittest.so")
 LIB_ROLES = os.path.join(HERE, "libfp8moe_roles.so")
 VARIANTS = {LIB: [], LIB_WAITTEST: ["-DMOE_WAIT_TEST"], LIB_ROLES: ["-DMOE_ROLE_COUNTERS"]}
 SOURCES = ["moe_api.cu", "route.cu", "router_mma.cu", "permute.cu", "gemm.cu", "combine.cu",
-           "noalloc.cu"]
+           "noalloc.cu", "dispatch.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -27,7 +27,7 @@ constexpr int kStatusDeviceCheck = -6;
 // where-codes stored next to the status (ws int[1]) to tell which kernel reported it
 enum Where : int {
   kWhereRoute = 1, kWherePermute = 2, kWhereGather = 3, kWhereGemm1 = 4, kWhereRequant = 5,
-  kWhereGemm2 = 6, kWhereCombine = 7, kWhereTilePrefix = 8,
+  kWhereGemm2 = 6, kWhereCombine = 7, kWhereTilePrefix = 8, kWhereDispatch = 9,
 };
 
 __device__ __forceinline__ void report(int* status, int code, int where, int detail) {

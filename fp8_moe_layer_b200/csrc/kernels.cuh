@@ -172,6 +172,18 @@ cudaError_t launch_combine(const Plan& p, const float* o, int splits, size_t spl
 cudaError_t launch_reduce_splits(const Plan& p, const float* o, int splits, size_t split_stride,
                                  const int32_t* total_rows, float* out, cudaStream_t s);
 
+// Expert-parallel dispatch over n_ranks contiguous expert blocks: plan (send rows in (rank,
+// token) order, local ids and weights, per-rank counts, the combine map) and the row gather.
+__host__ __device__ inline int ep_local_k(int E, int k_max, int n_ranks) {
+  const int el = E / n_ranks;
+  return k_max < el ? k_max : el;
+}
+cudaError_t launch_ep_dispatch(const Plan& p, int n_ranks, const uint16_t* hidden,
+                               const int32_t* ids, const float* topk_w, int k,
+                               const int32_t* k_per_token, uint16_t* send_hidden,
+                               int32_t* send_ids, float* send_w, int32_t* send_counts,
+                               int32_t* slot_of, float* slot_w, int* status, cudaStream_t s);
+
 int num_sms();
 
 }  // namespace moe

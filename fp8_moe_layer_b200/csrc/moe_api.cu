@@ -697,4 +697,33 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
   return MOE_OK;
 }
 
+int moe_ep_dispatch(const moe_dims* dims, int32_t n_ranks, const uint16_t* hidden,
+                    const int32_t* topk_ids, const float* topk_w, int32_t k,
+                    const int32_t* k_per_token, uint16_t* send_hidden, int32_t* send_ids,
+                    float* send_w, int32_t* send_counts, int32_t* slot_of, float* slot_w,
+                    void* ws, size_t ws_bytes, void* stream) {
+  if (!dims) return MOE_ERR_INVALID_ARG;
+  Plan p;
+  MOE_TRY(plan_make(dims->T, dims->d, dims->E, dims->F, dims->k_max, dims->F_shared, &p));
+  if (n_ranks < 1 || n_ranks > 32 || p.E % n_ranks != 0) return MOE_ERR_INVALID_ARG;
+  if (!send_counts) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p.T == 0) {
+    MOE_TRY(check_device());
+    MOE_CUDA(cudaMemsetAsync(send_counts, 0, sizeof(int32_t) * n_ranks, s));
+    return MOE_OK;
+  }
+  if (!hidden || !topk_ids || !topk_w || !send_hidden || !send_ids || !send_w || !slot_of ||
+      !slot_w)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(send_hidden, 16)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_k(p, k, k_per_token));
+  MOE_TRY(check_ws(p, ws, ws_bytes));
+  MOE_TRY(check_device());
+  Ws w = carve(p, ws);
+  MOE_CUDA(launch_ep_dispatch(p, n_ranks, hidden, topk_ids, topk_w, k, k_per_token, send_hidden,
+                              send_ids, send_w, send_counts, slot_of, slot_w, w.status, s));
+  return MOE_OK;
+}
+
 }  // extern "C"

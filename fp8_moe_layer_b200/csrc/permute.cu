@@ -77,7 +77,7 @@ __device__ int permute_block_body(const int32_t* __restrict__ ids, int T, int k_
       if (j < kt) {
         const int e = ids[idx];
         if (e >= 0 && e < E) atomicAdd(&my_hist[e], 1);
-        else if (write) report(status, kStatusDeviceCheck, kWherePermute, t);
+        else if (write && e != -1) report(status, kStatusDeviceCheck, kWherePermute, t);
       }
     }
   }
@@ -242,7 +242,7 @@ __device__ __forceinline__ void block_warp_counts(const int32_t* ids, int T, int
       if (j < kt) {
         const int e = ids[idx];
         if (e >= 0 && e < E) atomicAdd(&my[e], 1);
-        else if (flag) report(status, kStatusDeviceCheck, kWherePermute, t);
+        else if (flag && e != -1) report(status, kStatusDeviceCheck, kWherePermute, t);
       }
     }
   }

@@ -68,6 +68,8 @@ def _load(path: str = LIB_PATH) -> ctypes.CDLL:
                                        vp, vp, vp, sz, vp, ctypes.POINTER(MoEDebugOut)]),
         "moe_route_topk_noalloc": (ctypes.c_int, [dims_p, vp, vp, vp, i32, vp, vp, vp, vp]),
         "moe_kernel_launch_count": (ctypes.c_uint64, []),
+        "moe_ep_dispatch": (ctypes.c_int, [dims_p, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
+                                           vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -220,6 +222,38 @@ def moe_combine(expert_out, topk_w, inv_row, shared_out=None, want_f32=False):
                            _p(shared_out), _p(y.view(torch.int16)), _p(yf), _stream(dev)),
            "moe_combine")
     return (y, yf) if want_f32 else y
+
+
+def ep_local_k(E: int, k_max: int, n_ranks: int) -> int:
+    """Expert slots per dispatched row: a token has at most min(k_max, E / n_ranks) experts on
+    one rank."""
+    return min(k_max, E // n_ranks)
+
+
+def moe_ep_dispatch(hidden, topk_ids, topk_w, k, k_per_token, E, n_ranks, ws=None):
+    """Expert-parallel dispatch plan and row gather. Returns a dict: send_hidden bf16
+    [T*min(n_ranks, k_max), d], send_ids int32 / send_w fp32 [same rows, kl], send_counts int32
+    [n_ranks] (device), slot_of int32 / slot_w fp32 [T, n_ranks]."""
+    T, d = hidden.shape
+    k_max = topk_ids.shape[1]
+    dev = hidden.device
+    dm = dims(T, d, E, 16, k_max)
+    kl = ep_local_k(E, k_max, n_ranks)
+    cap = max(T * min(n_ranks, k_max), 1)
+    out = dict(send_hidden=torch.empty(cap, d, dtype=torch.bfloat16, device=dev),
+               send_ids=torch.empty(cap, kl, dtype=torch.int32, device=dev),
+               send_w=torch.empty(cap, kl, dtype=torch.float32, device=dev),
+               send_counts=torch.empty(n_ranks, dtype=torch.int32, device=dev),
+               slot_of=torch.empty(max(T, 1), n_ranks, dtype=torch.int32, device=dev),
+               slot_w=torch.empty(max(T, 1), n_ranks, dtype=torch.float32, device=dev))
+    ws = alloc_workspace(dims(max(T, 1), d, E, 16, k_max), dev) if ws is None else ws
+    _check(LIB.moe_ep_dispatch(ctypes.byref(dm), int(n_ranks), _p(_bits(hidden)), _p(topk_ids),
+                               _p(topk_w), int(k), _p(k_per_token),
+                               _p(out["send_hidden"].view(torch.int16)), _p(out["send_ids"]),
+                               _p(out["send_w"]), _p(out["send_counts"]), _p(out["slot_of"]),
+                               _p(out["slot_w"]), _p(ws), ws.numel(), _stream(dev)),
+           "moe_ep_dispatch")
+    return out
 
 
 def moe_forward(hidden, router_w, router_bias, k, k_per_token, w13, w13_scale, w2, w2_scale,

@@ -128,7 +128,8 @@ int moe_route_topk(const moe_dims* dims, const uint16_t* hidden, const float* ro
  *   out expert_offsets [E+1] int32 (offsets[E] = R = number of routed rows),
  *       perm_token [T*k_max] int32 (token of routed row r, r < R),
  *       inv_row [T, k_max] int32 (routed row of (t, j); -1 for unused slots).
- * An expert id outside [0, E) is skipped and flags MOE_ERR_DEVICE_CHECK. */
+ * An id of -1 marks an unused slot (as the expert-parallel receiver pads its rows); any other
+ * expert id outside [0, E) is skipped and flags MOE_ERR_DEVICE_CHECK. */
 int moe_permute(const moe_dims* dims, const int32_t* topk_ids, int32_t k,
                 const int32_t* k_per_token, int32_t* expert_offsets, int32_t* perm_token,
                 int32_t* inv_row, void* ws, size_t ws_bytes, void* stream);
@@ -193,6 +194,37 @@ int moe_forward(const moe_dims* dims, const uint16_t* hidden, const float* route
 int moe_route_topk_noalloc(const moe_dims* dims, const uint16_t* hidden, const float* router_w,
                            const float* router_bias, int32_t k, const int32_t* k_per_token,
                            int32_t* topk_ids, float* topk_w, void* stream);
+
+/* Expert-parallel dispatch ("Routage MoE entre GPU": a token's activations are sent to the GPUs
+ * that hold its selected experts and the results are sent back; "Semantic Parallelism", section 1:
+ * the all-to-all exchange of expert parallelism). The E experts are split over n_ranks GPUs in
+ * contiguous blocks of E_local = E / n_ranks: rank r holds experts [r * E_local, (r+1) * E_local).
+ * For every token t and every rank r that holds at least one of t's selected experts, one send
+ * row is written; the rows are ordered by (rank ascending, token ascending), so the rows for rank
+ * r are one contiguous segment of send_counts[r] rows. With kl = min(k_max, E_local):
+ *   dims: T, d, E, k_max as for moe_route_topk (F must be valid; F_shared is ignored);
+ *   n_ranks in [1, 32], dividing E;
+ *   hidden [T, d] bf16; topk_ids, topk_w [T, k_max] (the output of moe_route_topk); k /
+ *   k_per_token as in moe_permute;
+ *   out send_hidden [T * min(n_ranks, k_max), d] bf16 (capacity; rows >= sum(send_counts) are
+ *       untouched): send row i holds the hidden row of its token;
+ *       send_ids [same rows, kl] int32: the local ids (e - r * E_local) of the token's experts on
+ *       rank r in slot order, then -1;  send_w [same rows, kl] fp32: their routing weights, then 0;
+ *       send_counts [n_ranks] int32: rows for each rank (also written when T == 0);
+ *       slot_of [T, n_ranks] int32: the send row of (t, r), or -1;
+ *       slot_w [T, n_ranks] fp32: 1 where slot_of >= 0, else 0.
+ * On rank r the segment it receives from every source is a batch of tokens with kl local experts
+ * each (-1 = unused slot): moe_permute, moe_grouped_ffn_fp8 and moe_combine (its y_f32 output,
+ * E = E_local, k_max = kl) give the partial outputs, which go back to the sources in the same row
+ * order; there moe_combine with k_max = n_ranks, inv_row = slot_of, topk_w = slot_w and the shared
+ * expert's output as shared_out sums them into y. hidden and send_hidden must be 16-byte aligned;
+ * ws as for the other entry points (its status word). An expert id >= E, a k_t outside [0, k_max]
+ * or an expert selected twice for one token flags MOE_ERR_DEVICE_CHECK. */
+int moe_ep_dispatch(const moe_dims* dims, int32_t n_ranks, const uint16_t* hidden,
+                    const int32_t* topk_ids, const float* topk_w, int32_t k,
+                    const int32_t* k_per_token, uint16_t* send_hidden, int32_t* send_ids,
+                    float* send_w, int32_t* send_counts, int32_t* slot_of, float* slot_w,
+                    void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

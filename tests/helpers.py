@@ -180,3 +180,31 @@ def check_output(y_bf16: torch.Tensor, y_f32, y64: np.ndarray, what=""):
     assert np.all(err_b <= Y_ATOL + bf16_half_ulp(y64)), (what, stats)
     assert stats["rel_l2"] <= Y_REL_L2, (what, stats)
     return stats
+
+
+def ep_dispatch_reference(ids: np.ndarray, w: np.ndarray, k_t: np.ndarray, E: int, n_ranks: int):
+    """The expert-parallel send plan written out with loops: one row per (rank, token) pair where
+    the rank holds one of the token's selected experts, rows ordered by rank then token; a row's
+    local ids (global id - rank * E/n) and weights in slot order, padded with -1 / 0 to
+    kl = min(k_max, E/n) slots."""
+    T, k_max = ids.shape
+    El = E // n_ranks
+    kl = min(k_max, El)
+    tokens, rids, rw = [], [], []
+    counts = np.zeros(n_ranks, dtype=np.int64)
+    slot_of = np.full((T, n_ranks), -1, dtype=np.int32)
+    for r in range(n_ranks):
+        for t in range(T):
+            sel = [j for j in range(int(k_t[t])) if r * El <= ids[t, j] < (r + 1) * El]
+            if not sel:
+                continue
+            slot_of[t, r] = len(tokens)
+            tokens.append(t)
+            rids.append([int(ids[t, j]) - r * El for j in sel] + [-1] * (kl - len(sel)))
+            rw.append([float(w[t, j]) for j in sel] + [0.0] * (kl - len(sel)))
+            counts[r] += 1
+    return dict(tokens=np.array(tokens, dtype=np.int64),
+                send_ids=np.array(rids, dtype=np.int32).reshape(-1, kl),
+                send_w=np.array(rw, dtype=np.float32).reshape(-1, kl),
+                counts=counts, slot_of=slot_of,
+                slot_w=(slot_of >= 0).astype(np.float32), kl=kl)

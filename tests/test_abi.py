@@ -76,6 +76,20 @@ def test_host_validation_without_gpu(ops):
                             None) == ops.MOE_ERR_INVALID_ARG
     assert L.moe_route_topk(ctypes.byref(dm), fake, fake, None, 2, None, fake, fake, fake, 16,
                             None) == ops.MOE_ERR_WORKSPACE
+    # expert-parallel dispatch: the rank count must divide E and lie in [1, 32]
+    ep = lambda dm_, n, k, ws_bytes, cnt=fake: L.moe_ep_dispatch(
+        ctypes.byref(dm_), n, fake, fake, fake, k, None, fake, fake, fake, cnt, fake, fake, fake,
+        ws_bytes, None)
+    assert ep(dm, 3, 2, 1 << 30) == ops.MOE_ERR_INVALID_ARG
+    assert ep(dm, 0, 2, 1 << 30) == ops.MOE_ERR_INVALID_ARG
+    assert ep(ops.dims(4, 128, 64, 256, 2), 64, 2, 1 << 30) == ops.MOE_ERR_INVALID_ARG
+    assert ep(dm, 4, 2, 1 << 30, cnt=None) == ops.MOE_ERR_INVALID_ARG
+    assert ep(dm, 4, 3, 1 << 30) == ops.MOE_ERR_INVALID_ARG          # k > k_max
+    assert ep(dm, 4, 2, 16) == ops.MOE_ERR_WORKSPACE
+    assert ep(bad, 4, 2, 1 << 30) == ops.MOE_ERR_INVALID_ARG
+    assert L.moe_ep_dispatch(ctypes.byref(dm), 4, ctypes.c_void_p((1 << 20) + 8), fake, fake, 2,
+                             None, fake, fake, fake, fake, fake, fake, fake, 1 << 30,
+                             None) == ops.MOE_ERR_INVALID_ARG              # hidden misaligned
     # T == 0 is a valid no-op
     zero = ops.dims(0, 128, 8, 256, 2)
     assert L.moe_forward(ctypes.byref(zero), *([None] * 3), 2, *([None] * 11), 0, None,
@@ -106,6 +120,9 @@ SIGNATURES = {
                    "size_t, void*, const moe_debug_out*)",
     "moe_route_topk_noalloc": "int (*)(const moe_dims*, const uint16_t*, const float*, "
                               "const float*, int32_t, const int32_t*, int32_t*, float*, void*)",
+    "moe_ep_dispatch": "int (*)(const moe_dims*, int32_t, const uint16_t*, const int32_t*, "
+                       "const float*, int32_t, const int32_t*, uint16_t*, int32_t*, float*, "
+                       "int32_t*, int32_t*, float*, void*, size_t, void*)",
 }
 
 

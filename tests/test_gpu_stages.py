@@ -98,6 +98,24 @@ def test_permute_flags_out_of_range_expert_ids(ops):
     assert H.np_(offsets)[E] == 2 * T - 1 and H.np_(inv)[3, 1] == -1
 
 
+def test_permute_skips_unused_slots_without_a_report(ops):
+    """-1 inside a token's k_t slots is an unused slot (the expert-parallel receiver's padding):
+    skipped, not reported."""
+    T, E, k_max = 10, 4, 3
+    ids = np.tile(np.array([[2, 0, -1]], dtype=np.int32), (T, 1))
+    ids[4] = [-1, -1, 3]
+    dm = ops.dims(T, 16, E, 16, k_max)
+    ws = ops.alloc_workspace(dm)
+    offsets, perm, inv = ops.moe_permute(torch.from_numpy(ids).cuda(), k_max, None, E, ws=ws)
+    assert ops.device_status(ws) == ops.MOE_OK
+    pairs = sorted((int(ids[t, j]), t, j) for t in range(T) for j in range(k_max) if ids[t, j] >= 0)
+    assert H.np_(offsets).tolist() == [sum(1 for p in pairs if p[0] < e) for e in range(E + 1)]
+    assert H.np_(perm)[:len(pairs)].tolist() == [t for _, t, _ in pairs]
+    inv = H.np_(inv)
+    assert all(inv[t, j] == r for r, (_, t, j) in enumerate(pairs))
+    assert (inv[ids < 0] == -1).all()
+
+
 FFN_SHAPES = [
     I.WORKLOADS["tiny_T16"],
     I.MoEShape("ragged_K", 29, 192, 5, 96, 2, 2),        # K = 192, F = 96: partial tiles
