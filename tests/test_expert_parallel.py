@@ -152,3 +152,25 @@ def test_forward_orchestration_over_gloo(built, tmp_path, n):
     mp.start_processes(_worker, args=(n, _free_port(), str(tmp_path)), nprocs=n,
                        start_method="spawn")
     assert sorted(os.listdir(tmp_path)) == [f"ok{r}" for r in range(n)]
+
+
+@pytest.mark.parametrize("n,Ts", [(3, (9, 0, 14)), (1, (6,)), (5, (1, 2, 3, 4, 5))])
+def test_loopback_exchange_with_stand_in_ranks(built, n, Ts):
+    """loopback_forward's segment bookkeeping (who receives which rows, where the partial sums go
+    back) on the CPU, with the same stand-in arithmetic as the gloo test."""
+    from fp8_moe_layer_b200 import expert_parallel as EP
+    E, k_max, d = 4 * n, 3, 8
+    ranks, xs, want = [], [], []
+    for r, T in enumerate(Ts):
+        layer = _stand_in_rank(EP, r, n, E, k_max, d)
+        ids, w, k_t = _routing(T, E, k_max, seed=50 + r, elastic=True)
+        layer.routing = (ids, w, k_t)
+        x = torch.from_numpy(np.random.default_rng(7 + r).standard_normal((T, d)))
+        coef = 0.5 + np.array([sum(float(w[t, j]) * (int(ids[t, j]) + 1) for j in range(k_t[t]))
+                               for t in range(T)])
+        ranks.append(layer)
+        xs.append(x)
+        want.append(coef[:, None] * x.numpy())
+    ys = EP.loopback_forward(ranks, xs)
+    for y, wnt in zip(ys, want):
+        np.testing.assert_allclose(y.numpy(), wnt, rtol=1e-6, atol=1e-12)
