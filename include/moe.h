@@ -218,8 +218,9 @@ int moe_route_topk_noalloc(const moe_dims* dims, const uint16_t* hidden, const f
  * E = E_local, k_max = kl) give the partial outputs, which go back to the sources in the same row
  * order; there moe_combine with k_max = n_ranks, inv_row = slot_of, topk_w = slot_w and the shared
  * expert's output as shared_out sums them into y. hidden and send_hidden must be 16-byte aligned;
- * ws as for the other entry points (its status word). An expert id >= E, a k_t outside [0, k_max]
- * or an expert selected twice for one token flags MOE_ERR_DEVICE_CHECK. */
+ * ws: at least moe_workspace_bytes(dims) bytes, as for the other entry points (only its status
+ * word is used). An expert id >= E, a k_t outside [0, k_max] or an expert selected twice for one
+ * token flags MOE_ERR_DEVICE_CHECK; such ids are left out of the plan. */
 int moe_ep_dispatch(const moe_dims* dims, int32_t n_ranks, const uint16_t* hidden,
                     const int32_t* topk_ids, const float* topk_w, int32_t k,
                     const int32_t* k_per_token, uint16_t* send_hidden, int32_t* send_ids,
